@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 quantized linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = forward + backward of every QLoRA linear of a LLaMA-7B
+transformer block (q, k, v, o 4096x4096; gate, up 11008x4096; down
+4096x11008; 4096 tokens = 2 x 2048; r = 64, alpha = 16), seeded synthetic
+data, weights already NF4-quantised and resident.  The linears are not
+chained (attention, SwiGLU and norms are not part of the measured path).
+Multi-GPU (torchrun): data parallel, every rank its own 4096 tokens (weak
+scaling), the adapter gradients all-reduced (sum) over NCCL once per step.
+
+Prints one JSON line (rank 0): whole-job algorithmic TFLOP/s of the step
+(4 M K N + 6 M r (K + N) per linear; no dequantisation work counted), plus
+  e2e        same metric through the C ABI with the step's activations
+             copied host->device and the adapter gradients device->host
+             inside the timed region;
+  roofline   the fused dequant-GEMM launches (Y of the forward, dX of the
+             backward), timed live by events the library records around
+             them, against the measured sustained dense-bf16 peak;
+  quant / dequant   NF4 double-quantise and dequantise GB/s of the block's
+             7 weights against the measured HBM copy bandwidth;
+  cpu_baseline   the CPU oracle on a bounded sample of the same workload.
+`--impl reference` times that oracle as the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("fused QLoRA linear fwd+bwd TFLOP/s and % of roofline; "
+          "NF4 (de)quant GB/s vs HBM peak")
+WORKLOAD = "llama7b_block"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def linear_flops(M, N, K, r):
+    return 4.0 * M * K * N + 6.0 * M * r * (K + N)
+
+
+def main_gemm_flops(M, N, K, r):
+    # Y = X.W^T + (sT).L2 and dX = dY.W + (s dT).L1^T: the two fused launches
+    return (2.0 * M * K * N + 2.0 * M * r * N) + (2.0 * M * K * N + 2.0 * M * r * K)
+
+
+def quant_bytes(N, K):
+    n = N * K
+    return 2 * n + n // 2 + n // 64 + 4 * ((n // 64 + 255) // 256)
+
+
+def dequant_bytes(N, K):
+    n = N * K
+    return n // 2 + n // 64 + 4 * ((n // 64 + 255) // 256) + 2 * n
+
+
+# ----------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample_step(state):
+    """One bounded oracle step: dequantise the q-projection weight and run the
+    fp64 forward and backward of that linear on a sample of tokens."""
+    import oracle as O
+    codes, c2, c1, N, K, X, L1, L2, dY, s = state
+    What = O.bf16_bits_to_f64(O.dequant(codes, c2, c1, N, K))
+    Y, T = O.linear_fwd(X, What, L1, L2, s)
+    O.linear_bwd(dY, X, What, L1, L2, s, T)
+
+
+def oracle_state(tokens: int):
+    import numpy as np
+    import oracle as O
+    from bit_nf4_quantized_15_b200 import workloads as WL
+    wl = WL.WORKLOADS[WORKLOAD]
+    lin = wl.linears[0]
+    t = WL.make_linear(wl, lin, seed=0, device="cpu", M=tokens)
+    b = lambda x: WL.bf16_bits(x)
+    Wb = b(t["W"])
+    codes, c2, c1 = O.quantize(Wb)
+    X, L1, L2, dY = (O.bf16_bits_to_f64(b(t[k])) for k in ("X", "L1", "L2", "dY"))
+    return (codes, c2, c1, lin.N, lin.K, X, L1, L2, dY, wl.s), linear_flops(tokens, lin.N, lin.K, wl.r)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(tokens=256, reps=3):
+    state, flops = oracle_state(tokens)
+    oracle_sample_step(state)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle_sample_step(state)
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"q-projection 4096x4096 of {WORKLOAD}, {tokens} tokens, r=64: NF4 dequantise of the "
+                       f"weight + fp64 forward + backward, numpy on the host, mean of {reps} reps"),
+            "seconds_per_sample": dt}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    tokens = 128
+    state, flops = oracle_state(tokens)
+    for _ in range(args.warmup):
+        oracle_sample_step(state)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(state)
+    dt = time.perf_counter() - t0
+    v = flops * args.steps / dt / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_tokens": tokens, "linear": "q 4096x4096", "r": 64, "alpha": 16},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"q-projection of {WORKLOAD}, {tokens} tokens per step: dequantise + fp64 fwd + bwd"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import bit_nf4_quantized_15_b200 as q
+    from bit_nf4_quantized_15_b200 import workloads as WL
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = WL.WORKLOADS[args.workload]
+    M, r, s = wl.M, wl.r, wl.s
+    layers = []
+    max_ws = 0
+    for i, lin in enumerate(wl.linears):
+        t = WL.make_linear(wl, lin, seed=i, device=dev)
+        w = q.quantize(t["W"])
+        layers.append(dict(lin=lin, Wbf16=t["W"], w=w, X=t["X"], dY=t["dY"], L1=t["L1"], L2=t["L2"],
+                           Y=torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev),
+                           T=torch.empty((M, r), dtype=torch.float32, device=dev),
+                           dX=torch.empty((M, lin.K), dtype=torch.bfloat16, device=dev)))
+        max_ws = max(max_ws, q.workspace_bytes(M, lin.N, lin.K, r))
+    # adapter gradients of the block live in one flat buffer (one all-reduce per step)
+    sizes = [lin.K * r + r * lin.N for lin in wl.linears]
+    grads = torch.empty(sum(sizes), dtype=torch.float32, device=dev)
+    off = 0
+    for L, lin in zip(layers, wl.linears):
+        L["dL1"] = grads[off:off + lin.K * r].view(lin.K, r)
+        L["dL2"] = grads[off + lin.K * r:off + lin.K * r + r * lin.N].view(r, lin.N)
+        off += lin.K * r + r * lin.N
+    ws = torch.empty(max_ws, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    assert q.read_status(dev) == 0
+
+    n_lin = len(layers)
+    # per step, per linear: events around the forward and the backward fused dequant-GEMM
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_lin)]
+          for _ in range(args.steps)]
+    for es in ev:
+        for e4 in es:
+            for e in e4:
+                e.record()
+
+    def step(timed=None):
+        for i, L in enumerate(layers):
+            if timed is not None:
+                q.set_gemm_events(timed[i][0], timed[i][1])
+            q.linear_fwd(L["X"], L["w"], L["L1"], L["L2"], s, ws=ws, Y=L["Y"], T=L["T"])
+            if timed is not None:
+                q.set_gemm_events(timed[i][2], timed[i][3])
+            q.linear_bwd(L["dY"], L["X"], L["T"], L["w"], L["L1"], L["L2"], s, ws=ws,
+                         dX=L["dX"], dL1=L["dL1"], dL2=L["dL2"])
+        if world > 1:
+            import torch.distributed as dist
+            dist.all_reduce(grads)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    assert q.read_status(dev) == 0, "device status after warm-up"
+
+    # ---- timed region: device time of K steps, gemm events per launch
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    launches0 = q.kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    gemm_ms = 0.0
+    t0.record()
+    for k in range(args.steps):
+        step(timed=ev[k])
+    t1.record()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        for i in range(n_lin):
+            gemm_ms += ev[k][i][0].elapsed_time(ev[k][i][1]) + ev[k][i][2].elapsed_time(ev[k][i][3])
+    gemm_ms /= args.steps
+    launches = q.kernel_launches() - launches0
+    barrier(world)
+    clk = clocks.stop() if rank == 0 else None
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, world, dev)
+    assert q.read_status(dev) == 0, "device status after the timed region"
+
+    step_flops = sum(linear_flops(M, L["lin"].N, L["lin"].K, r) for L in layers)
+    value = step_flops * world * args.steps / (ms_max / 1e3) / 1e12
+    gemm_flops = sum(main_gemm_flops(M, L["lin"].N, L["lin"].K, r) for L in layers)
+    pk, pk_kind = peaks()
+    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
+
+    # ---- NF4 quantise / dequantise of the block's weights
+    qb = sum(quant_bytes(L["lin"].N, L["lin"].K) for L in layers)
+    db = sum(dequant_bytes(L["lin"].N, L["lin"].K) for L in layers)
+    Wdeq = [torch.empty((L["lin"].N, L["lin"].K), dtype=torch.bfloat16, device=dev) for L in layers]
+    wq = [q.NF4Weight.empty(L["lin"].N, L["lin"].K, dev) for L in layers]
+    for _ in range(2):
+        for L, o in zip(layers, wq):
+            q.quantize_into(L["Wbf16"], o)
+        for L, o in zip(layers, Wdeq):
+            q.dequant(L["w"], out=o)
+    torch.cuda.synchronize()
+    reps = max(args.steps, 3)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(reps):
+        for L, o in zip(layers, wq):
+            q.quantize_into(L["Wbf16"], o)
+    a1.record()
+    torch.cuda.synchronize()
+    quant_gbs = qb * reps / (a0.elapsed_time(a1) / 1e3) / 1e9
+    a0.record()
+    for _ in range(reps):
+        for L, o in zip(layers, Wdeq):
+            q.dequant(L["w"], out=o)
+    a1.record()
+    torch.cuda.synchronize()
+    dequant_gbs = db * reps / (a0.elapsed_time(a1) / 1e3) / 1e9
+    del Wdeq, wq
+    assert q.read_status(dev) == 0
+
+    # ---- end to end through the C ABI: activations in, adapter grads out
+    pin = lambda t: t.detach().cpu().pin_memory()
+    hX = [pin(L["X"]) for L in layers]
+    hdY = [pin(L["dY"]) for L in layers]
+    hG = torch.empty(grads.numel(), dtype=torch.float32, pin_memory=True)
+    h2d = sum(x.numel() * 2 + y.numel() * 2 for x, y in zip(hX, hdY))
+    d2h = grads.numel() * 4
+
+    def e2e_step():
+        for i, L in enumerate(layers):
+            L["X"].copy_(hX[i], non_blocking=True)
+            L["dY"].copy_(hdY[i], non_blocking=True)
+        step()
+        hG.copy_(grads, non_blocking=True)
+
+    for _ in range(max(args.warmup, 1)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = step_flops * world * args.steps / (e_ms / 1e3) / 1e12
+
+    if rank == 0:
+        base = cpu_baseline() if world == 1 and not args.no_cpu_baseline else None
+        hbm = pk["hbm_gbs"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "linears": [f"{l.name} {l.N}x{l.K}" for l in wl.linears],
+                       "tokens_per_gpu": M, "r": r, "alpha": wl.alpha, "global_tokens": M * world,
+                       "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2: each step streams ~0.7 GB of codes and activations",
+                       "tokens_per_s": M * world * args.steps / (ms_max / 1e3)},
+            "e2e": {"value": e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "roofline": {"bound": "tensor", "kernel": "fused dequant-GEMM (Y forward, dX backward)",
+                         "achieved": achieved, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops_sustained"], "traffic": None,
+                         "peak_source": f"{pk_kind} sustained dense bf16",
+                         "launches_timed": 2 * n_lin, "ms_per_launch": gemm_ms / (2 * n_lin)},
+            "quant": {"value": quant_gbs, "unit": "GB/s", "frac": quant_gbs / hbm, "peak": hbm,
+                      "bytes": qb, "peak_source": f"{pk_kind} HBM copy"},
+            "dequant": {"value": dequant_gbs, "unit": "GB/s", "frac": dequant_gbs / hbm, "peak": hbm,
+                        "bytes": db, "peak_source": f"{pk_kind} HBM copy"},
+            "cpu_baseline": base,
+            "clocks": clk,
+            "gpu_launches": launches,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,250 @@
-"""QLoRA NF4 quantized linear for NVIDIA B200 (sm_100a)."""
+"""QLoRA NF4 quantized linear layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libqlora_nf4.so`` (declared in
+``include/qlora_nf4.h``).  It only marshals arguments: every step of the
+computation runs in the library's CUDA kernels.  PyTorch is used for device
+memory and the current stream.  There is no CPU fallback: if the library
+is missing or the device is not sm_100, calls raise.
+
+    w = quantize(W)                       # NF4 double quantisation
+    What = dequant(w)                     # doubleDequant -> bf16
+    Y, T = linear_fwd(X, w, L1, L2, s)    # Y = X.W^T + s.X.L1.L2
+    dX, dL1, dL2 = linear_bwd(dY, X, T, w, L1, L2, s)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "lib", "NF4Weight", "quantize", "quantize_into", "dequant", "workspace_bytes", "linear_fwd", "linear_bwd",
+    "codebook", "status_string", "kernel_launches", "set_gemm_events", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
+
+QLORA_OK = 0
+QLORA_ERR_NONFINITE = -7
+QLORA_ERR_TIMEOUT = -8
+
+
+class QLoRAError(RuntimeError):
+    pass
+
+
+class qlora_nf4_weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p),
+                ("n_rows", ctypes.c_int64), ("n_cols", ctypes.c_int64)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGS = {
+    "qlora_nf4_storage_bytes": (ctypes.c_int, [_I64, _I64, ctypes.POINTER(ctypes.c_size_t),
+                                               ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "qlora_nf4_codebook": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float)]),
+    "qlora_nf4_quantize": (ctypes.c_int, [_P, _I64, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P]),
+    "qlora_nf4_dequant": (ctypes.c_int, [ctypes.POINTER(qlora_nf4_weight), _P, _P, _P]),
+    "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int]),
+    "qlora_linear_fwd": (ctypes.c_int, [_P, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P, ctypes.c_int,
+                                        ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _I64, _P, ctypes.POINTER(qlora_nf4_weight), _P, _P, ctypes.c_int,
+                                        ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qlora_kernel_launches": (ctypes.c_uint64, []),
+    "qlora_set_gemm_events": (ctypes.c_int, [_P, _P]),
+}
+
+
+def lib():
+    """The loaded C-ABI library (ctypes handle with typed entry points)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise QLoRAError(f"{LIB_PATH} is missing: build it with `python -m bit_nf4_quantized_15_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(h, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = h
+    return _lib
+
+
+def kernel_launches() -> int:
+    """Kernels launched through the library so far in this process."""
+    return int(lib().qlora_kernel_launches())
+
+
+def set_gemm_events(ev_start, ev_end):
+    """Record two torch.cuda.Event objects around the next call's fused
+    dequant-GEMM (diagnostic timing).  Both events must have been recorded
+    once already so that they exist."""
+    h0 = None if ev_start is None else ctypes.c_void_p(ev_start.cuda_event)
+    h1 = None if ev_end is None else ctypes.c_void_p(ev_end.cuda_event)
+    _check(lib().qlora_set_gemm_events(h0, h1))
+
+
+def status_string(code: int) -> str:
+    return lib().qlora_status_string(int(code)).decode()
+
+
+def _check(rc: int):
+    if rc != QLORA_OK:
+        raise QLoRAError(f"{status_string(rc)} (code {rc})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+_status_bufs = {}
+
+
+def _status(device) -> torch.Tensor:
+    idx = torch.device(device).index
+    if idx is None:
+        idx = torch.cuda.current_device()
+    buf = _status_bufs.get(idx)
+    if buf is None:
+        buf = torch.zeros(1, dtype=torch.int32, device=f"cuda:{idx}")
+        _status_bufs[idx] = buf
+    return buf
+
+
+def read_status(device="cuda") -> int:
+    """Synchronise, return and clear the device status word of `device`
+    (QLORA_OK or a QLORA_ERR_* the kernels reported)."""
+    buf = _status(device)
+    v = int(buf.item())
+    buf.zero_()
+    return v
+
+
+def _bf16_cuda(t, name):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise QLoRAError(f"{name} must be a contiguous bf16 CUDA tensor")
+    return t
+
+
+def storage_bytes(N: int, K: int):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().qlora_nf4_storage_bytes(N, K, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+@dataclass
+class NF4Weight:
+    """Quantized weight: codes uint8[N*K/2], c2 uint8[N*K/64] (E4M3), c1 float32[ceil(N*K/16384)]."""
+    codes: torch.Tensor
+    c2: torch.Tensor
+    c1: torch.Tensor
+    N: int
+    K: int
+
+    def descriptor(self) -> qlora_nf4_weight:
+        return qlora_nf4_weight(self.codes.data_ptr(), self.c2.data_ptr(), self.c1.data_ptr(), self.N, self.K)
+
+    @property
+    def device(self):
+        return self.codes.device
+
+    @staticmethod
+    def empty(N: int, K: int, device="cuda") -> "NF4Weight":
+        nc, n2, n1 = storage_bytes(N, K)
+        return NF4Weight(torch.empty(nc, dtype=torch.uint8, device=device),
+                         torch.empty(n2, dtype=torch.uint8, device=device),
+                         torch.empty(n1 // 4, dtype=torch.float32, device=device), N, K)
+
+
+def codebook():
+    arr = (ctypes.c_float * 16)()
+    _check(lib().qlora_nf4_codebook(arr))
+    return [float(v) for v in arr]
+
+
+def quantize_into(W: torch.Tensor, out: NF4Weight, status=None):
+    _bf16_cuda(W, "W")
+    N, K = W.shape
+    d = out.descriptor()
+    _check(lib().qlora_nf4_quantize(_ptr(W), N, K, ctypes.byref(d), _ptr(status if status is not None else _status(W.device)),
+                                    _stream(W.device)))
+    return out
+
+
+def quantize(W: torch.Tensor, status=None) -> NF4Weight:
+    """NF4 double quantisation of a bf16 CUDA weight [N, K] (K % 64 == 0)."""
+    _bf16_cuda(W, "W")
+    N, K = W.shape
+    return quantize_into(W, NF4Weight.empty(N, K, W.device), status)
+
+
+def dequant(w: NF4Weight, out: torch.Tensor | None = None, status=None) -> torch.Tensor:
+    """doubleDequant(c1, c2, W_NF4) -> bf16 [N, K]."""
+    if out is None:
+        out = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.device)
+    d = w.descriptor()
+    _check(lib().qlora_nf4_dequant(ctypes.byref(d), _ptr(out), _ptr(status if status is not None else _status(w.device)),
+                                   _stream(w.device)))
+    return out
+
+
+def workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    n = lib().qlora_workspace_bytes(M, N, K, r)
+    if n == 0:
+        raise QLoRAError("invalid shape or rank for qlora_workspace_bytes")
+    return n
+
+
+def _workspace(ws, M, N, K, r, device):
+    need = workspace_bytes(M, N, K, r)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def linear_fwd(X, w: NF4Weight, L1, L2, s: float, ws=None, Y=None, T=None, status=None):
+    """Y = X.W^T + s.(X.L1).L2 and T = X.L1 (fp32, for the backward)."""
+    _bf16_cuda(X, "X"), _bf16_cuda(L1, "L1"), _bf16_cuda(L2, "L2")
+    M, K = X.shape
+    r = L1.shape[1]
+    dev = X.device
+    Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=dev) if Y is None else Y
+    T = torch.empty((M, r), dtype=torch.float32, device=dev) if T is None else T
+    ws = _workspace(ws, M, w.N, w.K, r, dev)
+    d = w.descriptor()
+    _check(lib().qlora_linear_fwd(_ptr(X), M, ctypes.byref(d), _ptr(L1), _ptr(L2), r, float(s), _ptr(Y), _ptr(T),
+                                  _ptr(ws), ws.numel(), _ptr(status if status is not None else _status(dev)),
+                                  _stream(dev)))
+    return Y, T
+
+
+def linear_bwd(dY, X, T, w: NF4Weight, L1, L2, s: float, ws=None, need_dX=True, need_dL1=True, need_dL2=True,
+               status=None, dX=None, dL1=None, dL2=None):
+    """dX = dY.W^ + s.dT.L1^T, dL1 = s.X^T.dT, dL2 = s.T^T.dY (dT = dY.L2^T)."""
+    _bf16_cuda(dY, "dY"), _bf16_cuda(X, "X")
+    M, K = X.shape
+    r = L1.shape[1]
+    dev = X.device
+    if dX is None and need_dX:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if dL1 is None and need_dL1:
+        dL1 = torch.empty((K, r), dtype=torch.float32, device=dev)
+    if dL2 is None and need_dL2:
+        dL2 = torch.empty((r, w.N), dtype=torch.float32, device=dev)
+    ws = _workspace(ws, M, w.N, w.K, r, dev)
+    d = w.descriptor()
+    _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, _ptr(T), ctypes.byref(d), _ptr(L1), _ptr(L2), r, float(s),
+                                  _ptr(dX), _ptr(dL1), _ptr(dL2), _ptr(ws), ws.numel(),
+                                  _ptr(status if status is not None else _status(dev)), _stream(dev)))
+    return dX, dL1, dL2

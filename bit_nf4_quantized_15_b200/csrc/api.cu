@@ -1,0 +1,408 @@
+// The C ABI (include/qlora_nf4.h): argument checks, TMA tensor maps, the
+// launch plan of each call and the launches themselves.  No allocation, no
+// synchronisation: all work is queued on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qlora_nf4.h"
+#include "internal.h"
+
+using namespace qnf4;
+
+namespace {
+
+// --------------------------------------------------------------- device info
+struct DevInfo {
+  int ok = 0;
+  int sms = 148;
+};
+
+int current_device_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  static DevInfo cache[64];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (dev < 0 || dev >= 64) return QLORA_ERR_DEVICE;
+  if (!cache[dev].ok) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    if (major != 10 || minor != 0) return QLORA_ERR_DEVICE;
+    cache[dev].sms = sms;
+    cache[dev].ok = 1;
+  }
+  *out = cache[dev];
+  return QLORA_OK;
+}
+
+// ----------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major matrix [outer][inner] of `esize`-byte elements.
+int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t outer,
+             uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return QLORA_ERR_CUDA;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * (uint64_t)esize};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// bf16 operand of the engine.  K-major: matrix [mn][k] (k contiguous), box
+// 64 k x `rows` mn.  MN-major: matrix [k][mn] (mn contiguous), box 64 x 64.
+int map_operand(CUtensorMap* m, const void* base, int mn_major, uint64_t mn_extent, uint64_t k_extent, int rows) {
+  if (!mn_major)
+    return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_extent, mn_extent, 64, (uint32_t)rows,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, mn_extent, k_extent, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int map_codes(CUtensorMap* m, const uint8_t* codes, int64_t N, int64_t K, int mn_mode) {
+  // codes viewed as uint8 [N][K/2]
+  if (!mn_mode)
+    return make_map(m, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 32, 128,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  return make_map(m, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+EpiArgs epi_none() {
+  EpiArgs e;
+  std::memset(&e, 0, sizeof(e));
+  e.alpha = 1.0f;
+  e.alpha2 = 1.0f;
+  return e;
+}
+
+void fill_common(EngineArgs* a, int* status) {
+  std::memset(a, 0, sizeof(*a));
+  a->status = status;
+  const Nf4Tables& t = nf4_tables();
+  for (int i = 0; i < 16; ++i) a->q[i] = t.q[i];
+}
+
+// Launch the engine and, for a split reduction, the fixed-order sum.
+int run(EngineArgs& a, int amode, const GemmPlan& p, float* partial, cudaStream_t st) {
+  a.splits = p.splits;
+  a.partial = p.splits > 1 ? partial : nullptr;
+  if (launch_engine(a, amode, p, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (p.splits > 1 && launch_split_reduce(partial, p.splits, a.rows, a.cols, a.epi, st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Diagnostic events around the fused dequant-GEMM (qlora_set_gemm_events).
+cudaEvent_t g_ev_start = nullptr, g_ev_end = nullptr;
+
+int run_timed(EngineArgs& a, int amode, const GemmPlan& p, float* partial, cudaStream_t st) {
+  cudaEvent_t e0 = g_ev_start, e1 = g_ev_end;
+  g_ev_start = g_ev_end = nullptr;
+  if (e0 && cudaEventRecord(e0, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int rc = run(a, amode, p, partial, st);
+  if (rc == QLORA_OK && e1 && cudaEventRecord(e1, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  return rc;
+}
+
+bool valid_rank(int r) { return r >= 16 && r <= 128 && r % 16 == 0; }
+
+// Workspace layout shared by the forward and the backward:
+//   [0]             bf16 s.T   [M][r]
+//   [ofs_sdT]       bf16 s.dT  [M][r]
+//   [ofs_partial]   fp32 split partials of the largest split GEMM
+struct WsLayout {
+  size_t ofs_sdT, ofs_partial, total;
+  GemmPlan t_fwd, y_fwd, dt, dx, dl1, dl2;
+};
+
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
+  WsLayout w{};
+  const size_t mr = align256((size_t)M * r * 2);
+  w.ofs_sdT = mr;
+  w.ofs_partial = 2 * mr;
+  const int kbK = (int)(K / 64), kbN = (int)((N + 63) / 64), kbM = (int)((M + 63) / 64);
+  w.t_fwd = plan_gemm((int)M, r, kbK, sms);
+  w.y_fwd = plan_gemm((int)N, (int)M, kbK, sms);
+  w.dt = plan_gemm((int)M, r, kbN, sms);
+  w.dx = plan_gemm((int)K, (int)M, kbN, sms);
+  w.dl1 = plan_gemm((int)K, r, kbM, sms);
+  w.dl2 = plan_gemm((int)N, r, kbM, sms);
+  size_t part = 0;
+  for (const GemmPlan* p : {&w.t_fwd, &w.y_fwd, &w.dt, &w.dx, &w.dl1, &w.dl2})
+    part = p->partial_bytes > part ? p->partial_bytes : part;
+  w.total = w.ofs_partial + align256(part);
+  return w;
+}
+
+bool shape_ok(int64_t M, int64_t N, int64_t K) {
+  return M >= 1 && N >= 8 && K >= 64 && K % 64 == 0 && N % 8 == 0 && M <= (1 << 24) && N <= (1 << 24) &&
+         K <= (1 << 24);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qlora_status_string(int code) {
+  switch (code) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_NULL: return "a required pointer is NULL";
+    case QLORA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case QLORA_ERR_SHAPE: return "invalid shape (need K % 64 == 0, N % 8 == 0, sizes >= 1)";
+    case QLORA_ERR_RANK: return "unsupported LoRA rank (need r % 16 == 0, 16 <= r <= 128)";
+    case QLORA_ERR_WORKSPACE: return "workspace too small";
+    case QLORA_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case QLORA_ERR_NONFINITE: return "weight holds an Inf or NaN";
+    case QLORA_ERR_TIMEOUT: return "an internal GPU wait expired";
+    case QLORA_ERR_DEVICE: return "current device is not an sm_100 GPU";
+  }
+  return "unknown status";
+}
+
+int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes, size_t* c2_bytes, size_t* c1_bytes) {
+  if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
+  const int64_t n = N * K, nb = n / 64;
+  if (codes_bytes) *codes_bytes = (size_t)(n / 2);
+  if (c2_bytes) *c2_bytes = (size_t)nb;
+  if (c1_bytes) *c1_bytes = (size_t)((nb + 255) / 256) * 4;
+  return QLORA_OK;
+}
+
+uint64_t qlora_kernel_launches(void) { return launches_so_far(); }
+
+int qlora_set_gemm_events(void* ev_start, void* ev_end) {
+  g_ev_start = (ev_start && ev_end) ? reinterpret_cast<cudaEvent_t>(ev_start) : nullptr;
+  g_ev_end = (ev_start && ev_end) ? reinterpret_cast<cudaEvent_t>(ev_end) : nullptr;
+  return QLORA_OK;
+}
+
+int qlora_nf4_codebook(float levels[16]) {
+  if (!levels) return QLORA_ERR_NULL;
+  const Nf4Tables& t = nf4_tables();
+  for (int i = 0; i < 16; ++i) levels[i] = t.q[i];
+  return QLORA_OK;
+}
+
+int qlora_nf4_quantize(const uint16_t* W, int64_t N, int64_t K, const qlora_nf4_weight* out, int* status_dev,
+                       qlora_stream_t stream) {
+  if (!W || !out || !out->codes || !out->c2 || !out->c1) return QLORA_ERR_NULL;
+  if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(out->codes)) return QLORA_ERR_ALIGN;
+  DevInfo di;
+  if (int rc = current_device_info(&di)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch_quantize(W, N * K, out->codes, out->c2, out->c1, status_dev, st) == cudaSuccess ? QLORA_OK
+                                                                                                 : QLORA_ERR_CUDA;
+}
+
+int qlora_nf4_dequant(const qlora_nf4_weight* w, uint16_t* W_out, int* status_dev, qlora_stream_t stream) {
+  (void)status_dev;
+  if (!w || !W_out || !w->codes || !w->c2 || !w->c1) return QLORA_ERR_NULL;
+  if (w->n_rows < 1 || w->n_cols < 64 || w->n_cols % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(W_out) || !aligned16(w->codes)) return QLORA_ERR_ALIGN;
+  DevInfo di;
+  if (int rc = current_device_info(&di)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch_dequant(w->codes, w->c2, w->c1, w->n_rows * w->n_cols, W_out, st) == cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  if (!shape_ok(M, N, K) || !valid_rank(r)) return 0;
+  DevInfo di;
+  if (current_device_info(&di)) di.sms = 148;
+  return ws_layout(M, N, K, r, di.sms).total;
+}
+
+int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, const uint16_t* L1,
+                     const uint16_t* L2, int r, float s, uint16_t* Y, float* T_save, void* ws, size_t ws_bytes,
+                     int* status_dev, qlora_stream_t stream) {
+  if (!X || !w || !w->codes || !w->c2 || !w->c1 || !L1 || !L2 || !Y || !T_save || !ws) return QLORA_ERR_NULL;
+  const int64_t N = w->n_rows, K = w->n_cols;
+  if (!shape_ok(M, N, K)) return QLORA_ERR_SHAPE;
+  if (!valid_rank(r)) return QLORA_ERR_RANK;
+  for (const void* p : {(const void*)X, (const void*)w->codes, (const void*)L1, (const void*)L2, (const void*)Y,
+                        (const void*)T_save, (const void*)ws})
+    if (!aligned16(p)) return QLORA_ERR_ALIGN;
+  DevInfo di;
+  if (int rc = current_device_info(&di)) return rc;
+  const WsLayout lay = ws_layout(M, N, K, r, di.sms);
+  if (ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* sT = reinterpret_cast<uint16_t*>(wsb);
+  float* partial = reinterpret_cast<float*>(wsb + lay.ofs_partial);
+
+  // (1) T = X.L1 (fp32, saved) and s.T in bf16 for the LoRA extension.
+  {
+    EngineArgs a;
+    fill_common(&a, status_dev);
+    const GemmPlan& p = lay.t_fwd;
+    if (map_operand(&a.tmA, X, 0, M, K, 128) || map_operand(&a.tmB, L1, 1, r, K, p.BN)) return QLORA_ERR_CUDA;
+    a.rows = (int)M;
+    a.cols = r;
+    a.kb_main = (int)(K / 64);
+    a.b_mn_main = 1;
+    a.epi = epi_none();
+    a.epi.out = T_save;
+    a.epi.rs = r;
+    a.epi.cs = 1;
+    a.epi.out2 = sT;
+    a.epi.alpha2 = s;
+    a.epi.rs2 = r;
+    a.epi.cs2 = 1;
+    if (int rc = run(a, A_TMA, p, partial, st)) return rc;
+  }
+  // (2) Y^T = W^.X^T + L2^T.(s.T)^T, W^ dequantised on chip.
+  {
+    EngineArgs a;
+    fill_common(&a, status_dev);
+    const GemmPlan& p = lay.y_fwd;
+    if (map_codes(&a.tmA, w->codes, N, K, 0) || map_operand(&a.tmB, X, 0, M, K, p.BN) ||
+        map_operand(&a.tmAx, L2, 1, N, r, 128) || map_operand(&a.tmBx, sT, 0, M, r, p.BN))
+      return QLORA_ERR_CUDA;
+    a.c2 = w->c2;
+    a.c1 = w->c1;
+    a.wN = N;
+    a.wK = K;
+    a.rows = (int)N;
+    a.cols = (int)M;
+    a.kb_main = (int)(K / 64);
+    a.kb_ext = (r + 63) / 64;
+    a.a_mn_ext = 1;
+    a.epi = epi_none();
+    a.epi.out = Y;
+    a.epi.out_bf16 = 1;
+    a.epi.rs = 1;
+    a.epi.cs = N;
+    if (int rc = run_timed(a, A_DEQ_K, p, partial, st)) return rc;
+  }
+  return QLORA_OK;
+}
+
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const float* T_saved,
+                     const qlora_nf4_weight* w, const uint16_t* L1, const uint16_t* L2, int r, float s, uint16_t* dX,
+                     float* dL1, float* dL2, void* ws, size_t ws_bytes, int* status_dev, qlora_stream_t stream) {
+  if (!dY || !X || !T_saved || !w || !w->codes || !w->c2 || !w->c1 || !L1 || !L2 || !ws) return QLORA_ERR_NULL;
+  const int64_t N = w->n_rows, K = w->n_cols;
+  if (!shape_ok(M, N, K)) return QLORA_ERR_SHAPE;
+  if (!valid_rank(r)) return QLORA_ERR_RANK;
+  for (const void* p : {(const void*)dY, (const void*)X, (const void*)T_saved, (const void*)w->codes,
+                        (const void*)L1, (const void*)L2, (const void*)ws})
+    if (!aligned16(p)) return QLORA_ERR_ALIGN;
+  for (const void* p : {(const void*)dX, (const void*)dL1, (const void*)dL2})
+    if (p && !aligned16(p)) return QLORA_ERR_ALIGN;
+  DevInfo di;
+  if (int rc = current_device_info(&di)) return rc;
+  const WsLayout lay = ws_layout(M, N, K, r, di.sms);
+  if (ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* sT = reinterpret_cast<uint16_t*>(wsb);
+  uint16_t* sdT = reinterpret_cast<uint16_t*>(wsb + lay.ofs_sdT);
+  float* partial = reinterpret_cast<float*>(wsb + lay.ofs_partial);
+
+  // (0) s.T in bf16, the operand of dL2.
+  if (dL2 && launch_scale_to_bf16(T_saved, M * r, s, sT, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  // (1) dT = dY.L2^T, kept as s.dT in bf16.
+  {
+    EngineArgs a;
+    fill_common(&a, status_dev);
+    const GemmPlan& p = lay.dt;
+    if (map_operand(&a.tmA, dY, 0, M, N, 128) || map_operand(&a.tmB, L2, 0, r, N, p.BN)) return QLORA_ERR_CUDA;
+    a.rows = (int)M;
+    a.cols = r;
+    a.kb_main = (int)((N + 63) / 64);
+    a.epi = epi_none();
+    a.epi.out2 = sdT;
+    a.epi.alpha2 = s;
+    a.epi.rs2 = r;
+    a.epi.cs2 = 1;
+    if (int rc = run(a, A_TMA, p, partial, st)) return rc;
+  }
+  // (2) dX^T = W^T.dY^T + L1.(s.dT)^T, W^ dequantised on chip (MN-major).
+  if (dX) {
+    EngineArgs a;
+    fill_common(&a, status_dev);
+    const GemmPlan& p = lay.dx;
+    if (map_codes(&a.tmA, w->codes, N, K, 1) || map_operand(&a.tmB, dY, 0, M, N, p.BN) ||
+        map_operand(&a.tmAx, L1, 0, K, r, 128) || map_operand(&a.tmBx, sdT, 0, M, r, p.BN))
+      return QLORA_ERR_CUDA;
+    a.c2 = w->c2;
+    a.c1 = w->c1;
+    a.wN = N;
+    a.wK = K;
+    a.rows = (int)K;
+    a.cols = (int)M;
+    a.kb_main = (int)((N + 63) / 64);
+    a.kb_ext = (r + 63) / 64;
+    a.epi = epi_none();
+    a.epi.out = dX;
+    a.epi.out_bf16 = 1;
+    a.epi.rs = 1;
+    a.epi.cs = K;
+    if (int rc = run_timed(a, A_DEQ_MN, p, partial, st)) return rc;
+  }
+  // (3) dL1 = X^T.(s.dT): rows k, reduction over tokens.
+  if (dL1) {
+    EngineArgs a;
+    fill_common(&a, status_dev);
+    const GemmPlan& p = lay.dl1;
+    if (map_operand(&a.tmA, X, 1, K, M, 128) || map_operand(&a.tmB, sdT, 1, r, M, p.BN)) return QLORA_ERR_CUDA;
+    a.rows = (int)K;
+    a.cols = r;
+    a.kb_main = (int)((M + 63) / 64);
+    a.a_mn_main = 1;
+    a.b_mn_main = 1;
+    a.epi = epi_none();
+    a.epi.out = dL1;
+    a.epi.rs = r;
+    a.epi.cs = 1;
+    if (int rc = run(a, A_TMA, p, partial, st)) return rc;
+  }
+  // (4) dL2^T = dY^T.(s.T): rows n, reduction over tokens, stored as dL2[r][N].
+  if (dL2) {
+    EngineArgs a;
+    fill_common(&a, status_dev);
+    const GemmPlan& p = lay.dl2;
+    if (map_operand(&a.tmA, dY, 1, N, M, 128) || map_operand(&a.tmB, sT, 1, r, M, p.BN)) return QLORA_ERR_CUDA;
+    a.rows = (int)N;
+    a.cols = r;
+    a.kb_main = (int)((M + 63) / 64);
+    a.a_mn_main = 1;
+    a.b_mn_main = 1;
+    a.epi = epi_none();
+    a.epi.out = dL2;
+    a.epi.rs = 1;
+    a.epi.cs = N;
+    if (int rc = run(a, A_TMA, p, partial, st)) return rc;
+  }
+  return QLORA_OK;
+}
+
+}  // extern "C"

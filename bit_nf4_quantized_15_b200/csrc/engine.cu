@@ -1,0 +1,404 @@
+// The tcgen05 GEMM engine behind every contraction of the layer.
+//
+//   D[rows x cols] (fp32, in TMEM) = sum_k A[row, k] * B[col, k]
+//
+// One CTA computes a 128 x BN output tile with cta_group::1 UMMA (M = 128).
+// The reduction runs in 64-wide blocks through a 4-stage shared-memory ring:
+//   * warp 0, one lane: TMA producer (B tiles, A tiles or NF4 code tiles);
+//   * warp 1, one lane: UMMA issuer, 4 x (128 x BN x 16) MMAs per stage,
+//     tcgen05.commit frees the stage;
+//   * warps 2..5 (128 threads): when A is the NF4 weight, they turn the code
+//     tile into a bf16 tile in the 128-byte-swizzled canonical layout UMMA
+//     reads (K-major for X.W^T, MN-major for dY.W), then run the epilogue
+//     (TMEM -> registers -> global, one accumulator row per thread).
+// An optional extension segment appends more reduction blocks from other
+// operands into the same accumulator: this is how the LoRA term s.T.L2
+// (forward) and s.dT.L1^T (backward) is added to the dequantised product.
+// A split of the main reduction over grid.z writes fp32 partial tiles that
+// a second kernel sums in a fixed order (deterministic).
+//
+// inferensys glossary "QLoRA", kernel paragraph: 4-bit weights are loaded,
+// decompressed in shared memory and fed to the tensor cores as BFloat16.
+#include "common.cuh"
+#include "internal.h"
+
+namespace qnf4 {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kA = 16384;  // 128 rows x 64 bf16
+
+template <int BN>
+struct Tmem {
+  static constexpr uint32_t cols = BN < 32 ? 32 : BN;
+};
+
+template <int BN, int AMODE>
+struct Layout {
+  static constexpr int B = BN * 128 > 8192 ? BN * 128 : 8192;
+  static constexpr int C = AMODE == A_TMA ? 0 : 4096;
+  static constexpr int STAGE = kA + B + C;
+  static constexpr int BAR = kStages * STAGE;
+  static constexpr int TOTAL = BAR + 256 + 1024;  // barriers etc. + alignment slack
+};
+
+QDEV uint32_t tx_bytes(int mn_major, int extent) {
+  return mn_major ? (uint32_t)((extent + 63) / 64) * 8192u : (uint32_t)extent * 128u;
+}
+
+// Load one operand tile (extent rows of UMMA M/N, 64 of the reduction).
+QDEV void load_operand(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int mn_major, int mn0, int k0,
+                       int extent) {
+  if (!mn_major) {
+    tma_load_2d(dst, m, bar, k0, mn0);
+  } else {
+    for (int j = 0; j < (extent + 63) / 64; ++j) tma_load_2d(dst + j * 8192, m, bar, mn0 + 64 * j, k0);
+  }
+}
+
+QDEV uint64_t operand_desc(const uint8_t* base, int mn_major, int kk) {
+  const uint32_t a = smem_u32(base);
+  return mn_major ? sdesc_sw128(a + kk * 2048, 8192, 1024) : sdesc_sw128(a + kk * 32, 16, 1024);
+}
+
+QDEV void epi_store(const EpiArgs& e, int64_t row, int64_t col, float v) {
+  if (e.out) {
+    const int64_t i = row * e.rs + col * e.cs;
+    if (e.out_bf16) reinterpret_cast<__nv_bfloat16*>(e.out)[i] = __float2bfloat16_rn(__fmul_rn(v, e.alpha));
+    else reinterpret_cast<float*>(e.out)[i] = __fmul_rn(v, e.alpha);
+  }
+  if (e.out2) {
+    const int64_t i = row * e.rs2 + col * e.cs2;
+    reinterpret_cast<__nv_bfloat16*>(e.out2)[i] = __float2bfloat16_rn(__fmul_rn(v, e.alpha2));
+  }
+}
+
+template <int BN, int AMODE>
+__global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_constant__ EngineArgs args) {
+  using L = Layout<BN, AMODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR);
+  uint64_t* afull = full + kStages;
+  uint64_t* empty = afull + kStages;
+  uint64_t* accum = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* lut = reinterpret_cast<float*>(tmem_slot + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row0 = blockIdx.x * 128, col0 = blockIdx.y * BN, z = blockIdx.z;
+  const int kb_lo = (int)((int64_t)z * args.kb_main / args.splits);
+  const int kb_hi = (int)((int64_t)(z + 1) * args.kb_main / args.splits);
+  const int my_kb = kb_hi - kb_lo;
+  const int n_iters = my_kb + (z == 0 ? args.kb_ext : 0);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(afull + s, 4);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (tid < 16) lut[tid] = args.q[tid];
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&args.tmA);
+    tma_prefetch_desc(&args.tmB);
+    if (args.kb_ext) {
+      tma_prefetch_desc(&args.tmAx);
+      tma_prefetch_desc(&args.tmBx);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Tmem<BN>::cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  bool committed_accum = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
+        uint8_t* sa = smem + s * L::STAGE;
+        uint8_t* sb = sa + kA;
+        uint8_t* sc = sb + L::B;
+        if (it < my_kb) {
+          const int kb = kb_lo + it;
+          uint32_t bytes = tx_bytes(args.b_mn_main, BN);
+          bytes += AMODE == A_TMA ? tx_bytes(args.a_mn_main, 128) : 4096u;
+          mbar_arrive_expect_tx(full + s, bytes);
+          if (AMODE == A_DEQ_K) tma_load_2d(sc, &args.tmA, full + s, kb * 32, row0);
+          else if (AMODE == A_DEQ_MN) tma_load_2d(sc, &args.tmA, full + s, row0 / 2, kb * 64);
+          else load_operand(sa, &args.tmA, full + s, args.a_mn_main, row0, kb * 64, 128);
+          load_operand(sb, &args.tmB, full + s, args.b_mn_main, col0, kb * 64, BN);
+        } else {
+          const int kb = it - my_kb;
+          mbar_arrive_expect_tx(full + s, tx_bytes(args.a_mn_ext, 128) + tx_bytes(args.b_mn_ext, BN));
+          load_operand(sa, &args.tmAx, full + s, args.a_mn_ext, row0, kb * 64, 128);
+          load_operand(sb, &args.tmBx, full + s, args.b_mn_ext, col0, kb * 64, BN);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- UMMA
+    if (lane == 0) {
+      const int a_mn_main = AMODE == A_DEQ_MN ? 1 : (AMODE == A_DEQ_K ? 0 : args.a_mn_main);
+      const uint32_t id_main = idesc_bf16(128, BN, a_mn_main, args.b_mn_main);
+      const uint32_t id_ext = idesc_bf16(128, BN, args.a_mn_ext, args.b_mn_ext);
+      bool ok = true;
+      for (int it = 0; it < n_iters && ok; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const bool ext = it >= my_kb;
+        ok = mbar_wait(full + s, ph, abort_flag, args.status);
+        if (ok && AMODE != A_TMA && !ext) ok = mbar_wait(afull + s, ph, abort_flag, args.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint8_t* sa = smem + s * L::STAGE;
+        const uint8_t* sb = sa + kA;
+        const int amn = ext ? args.a_mn_ext : a_mn_main;
+        const int bmn = ext ? args.b_mn_ext : args.b_mn_main;
+        const uint32_t id = ext ? id_ext : id_main;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem_d, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (it | kk) != 0);
+        umma_commit(empty + s);
+      }
+      umma_commit(accum);
+      committed_accum = true;
+    }
+    __syncwarp();
+  } else {
+    const int e = tid - 64;  // 0..127
+    // ------------------------------------------------------------- dequant
+    if (AMODE == A_DEQ_K) {
+      // Thread e owns output row n = row0 + e (one NF4 block of 64 per stage).
+      const int64_t n = row0 + e;
+      const bool valid = n < args.wN;
+      const int64_t bpr = args.wK / 64;  // blocks per weight row
+      uint32_t c2raw = 0;
+      float c1v = 0.0f;
+      if (valid && my_kb > 0) {
+        const int64_t f = n * bpr + kb_lo;
+        c2raw = __ldg(args.c2 + f);
+        c1v = __ldg(args.c1 + (f >> 8));
+      }
+      const uint32_t swz = (uint32_t)(e & 7);
+      for (int it = 0; it < my_kb; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        if (valid && it + 1 < my_kb) {  // prefetch the next stage's scale
+          const int64_t f = n * bpr + kb_lo + it + 1;
+          c2raw = __ldg(args.c2 + f);
+          c1v = __ldg(args.c1 + (f >> 8));
+        }
+        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
+        if (!mbar_wait(full + s, ph, abort_flag, args.status)) break;
+        const uint8_t* sc = smem + s * L::STAGE + kA + L::B;
+        uint8_t* sa = smem + s * L::STAGE;
+        const uint4 cw0 = *reinterpret_cast<const uint4*>(sc + e * 32);
+        const uint4 cw1 = *reinterpret_cast<const uint4*>(sc + e * 32 + 16);
+        const uint32_t words[8] = {cw0.x, cw0.y, cw0.z, cw0.w, cw1.x, cw1.y, cw1.z, cw1.w};
+        uint8_t* rowp = sa + (e >> 3) * 1024 + (e & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // chunk c: k = 8c .. 8c+7
+          const uint32_t w = words[c];
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t b = w >> (8 * k);
+            o[k] = pack_bf16x2(__fmul_rn(lut[b & 15u], chat), __fmul_rn(lut[(b >> 4) & 15u], chat));
+          }
+          *reinterpret_cast<uint4*>(rowp + (((uint32_t)c ^ swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull + s);
+      }
+    } else if (AMODE == A_DEQ_MN) {
+      // A = W^T: rows are k (W columns), the reduction runs over n (W rows).
+      // Thread e: 16 consecutive k (w2 = e % 8 -> k_local = 16 w2) of rows
+      // n_local = e/8 + 16 i, i = 0..3.
+      const int w2 = e & 7, rg = e >> 3;
+      const int64_t bpr = args.wK / 64;
+      const int64_t kblk = (int64_t)(row0 >> 6) + (w2 >> 2);
+      const bool kvalid = kblk < bpr;
+      const int mb = w2 >> 2;
+      const uint32_t cA = (uint32_t)(2 * (w2 & 3));
+      const bool swap = w2 >= 4;  // store order that keeps an 8-thread phase conflict-free
+      for (int it = 0; it < my_kb; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const int64_t n0 = (int64_t)(kb_lo + it) * 64;
+        uint32_t c2r[4];
+        float c1r[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t n = n0 + rg + 16 * i;
+          c2r[i] = 0;
+          c1r[i] = 0.0f;
+          if (kvalid && n < args.wN) {
+            const int64_t f = n * bpr + kblk;
+            c2r[i] = __ldg(args.c2 + f);
+            c1r[i] = __ldg(args.c1 + (f >> 8));
+          }
+        }
+        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
+        if (!mbar_wait(full + s, ph, abort_flag, args.status)) break;
+        const uint8_t* sc = smem + s * L::STAGE + kA + L::B;
+        uint8_t* sa = smem + s * L::STAGE;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int nl = rg + 16 * i;
+          const float chat = (c1r[i] != 0.0f) ? decode_scale(c2r[i], c1r[i]) : 0.0f;
+          const uint2 cw = *reinterpret_cast<const uint2*>(sc + nl * 64 + w2 * 8);
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t b0 = cw.x >> (8 * k), b1 = cw.y >> (8 * k);
+            o[k] = pack_bf16x2(__fmul_rn(lut[b0 & 15u], chat), __fmul_rn(lut[(b0 >> 4) & 15u], chat));
+            o[4 + k] = pack_bf16x2(__fmul_rn(lut[b1 & 15u], chat), __fmul_rn(lut[(b1 >> 4) & 15u], chat));
+          }
+          const uint32_t r8 = (uint32_t)(nl & 7);
+          uint8_t* atom = sa + mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
+          const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]);
+          const uint4 hi = make_uint4(o[4], o[5], o[6], o[7]);
+          if (!swap) {
+            *reinterpret_cast<uint4*>(atom + ((cA ^ r8) << 4)) = lo;
+            *reinterpret_cast<uint4*>(atom + (((cA + 1) ^ r8) << 4)) = hi;
+          } else {
+            *reinterpret_cast<uint4*>(atom + (((cA + 1) ^ r8) << 4)) = hi;
+            *reinterpret_cast<uint4*>(atom + ((cA ^ r8) << 4)) = lo;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull + s);
+      }
+    }
+    // ------------------------------------------------------------ epilogue
+    const bool ok = mbar_wait(accum, 0, abort_flag, args.status);
+    tc_fence_after();
+    const int q4 = warp & 3;
+    const int64_t row = row0 + q4 * 32 + lane;
+    for (int c = 0; c < BN; c += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem_d + ((uint32_t)(q4 * 32) << 16) + (uint32_t)c, v);
+      tmem_wait_ld();
+      if (!ok || *abort_flag || row >= args.rows) continue;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t col = col0 + c + j;
+        if (col >= args.cols) break;
+        const float x = __uint_as_float(v[j]);
+        if (args.splits > 1) args.partial[((int64_t)z * args.cols + col) * args.rows + row] = x;
+        else epi_store(args.epi, row, col, x);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (*abort_flag && lane == 0 && committed_accum) mbar_wait_drain(accum, 0, 10000000ull);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_d, Tmem<BN>::cols);
+  }
+}
+
+__global__ void split_reduce_kernel(const float* __restrict__ partial, int splits, int rows, int cols, EpiArgs e) {
+  const int64_t total = (int64_t)rows * cols;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i % rows, col = i / rows;
+    float acc = 0.0f;
+    for (int z = 0; z < splits; ++z) acc += partial[((int64_t)z * cols + col) * rows + row];
+    epi_store(e, row, col, acc);
+  }
+}
+
+template <int BN, int AMODE>
+cudaError_t launch_t(const EngineArgs& a, const GemmPlan& p, cudaStream_t st) {
+  using L = Layout<BN, AMODE>;
+  auto kern = umma_engine_kernel<BN, AMODE>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+  if (err != cudaSuccess) return err;
+  dim3 grid(p.m_tiles, p.n_tiles, p.splits);
+  kern<<<grid, kThreads, L::TOTAL, st>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int AMODE>
+cudaError_t launch_mode(const EngineArgs& a, const GemmPlan& p, cudaStream_t st) {
+  switch (p.BN) {
+    case 16: return launch_t<16, AMODE>(a, p, st);
+    case 32: return launch_t<32, AMODE>(a, p, st);
+    case 64: return launch_t<64, AMODE>(a, p, st);
+    case 128: return launch_t<128, AMODE>(a, p, st);
+    case 256: return launch_t<256, AMODE>(a, p, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+int bn_for_cols(int cols) { return cols <= 16 ? 16 : cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : 256; }
+
+GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms) {
+  GemmPlan p{};
+  p.BN = bn_for_cols(cols);
+  p.m_tiles = (rows + 127) / 128;
+  p.n_tiles = (cols + p.BN - 1) / p.BN;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int target = num_sms * (p.BN <= 64 ? 2 : 1);
+  int splits = 1;
+  if (tiles < target) {
+    splits = (target + tiles - 1) / tiles;
+    const int cap = kb_main / 4 > 1 ? kb_main / 4 : 1;
+    if (splits > cap) splits = cap;
+    if (splits > 64) splits = 64;
+  }
+  p.splits = splits;
+  p.partial_bytes = splits > 1 ? (size_t)splits * rows * cols * sizeof(float) : 0;
+  return p;
+}
+
+size_t engine_smem_bytes(int BN, int amode) {
+  const int b = BN * 128 > 8192 ? BN * 128 : 8192;
+  const int c = amode == A_TMA ? 0 : 4096;
+  return (size_t)kStages * (kA + b + c) + 256 + 1024;
+}
+
+cudaError_t launch_engine(const EngineArgs& a, int amode, const GemmPlan& p, cudaStream_t st) {
+  switch (amode) {
+    case A_TMA: return launch_mode<A_TMA>(a, p, st);
+    case A_DEQ_K: return launch_mode<A_DEQ_K>(a, p, st);
+    case A_DEQ_MN: return launch_mode<A_DEQ_MN>(a, p, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_split_reduce(const float* partial, int splits, int rows, int cols, const EpiArgs& e,
+                                cudaStream_t st) {
+  const int64_t total = (int64_t)rows * cols;
+  const int64_t want = (total + 255) / 256;
+  const int grid = (int)(want < 4096 ? (want > 0 ? want : 1) : 4096);
+  split_reduce_kernel<<<grid, 256, 0, st>>>(partial, splits, rows, cols, e);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

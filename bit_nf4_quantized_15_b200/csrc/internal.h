@@ -1,0 +1,86 @@
+// Internal declarations shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qnf4 {
+
+// NF4 codebook and decision thresholds as the kernels use them.
+//   q[i] : the 16 levels (fp32), ascending, q[7] = 0 exactly.
+//   t[i] : RD32 of the exact midpoint (q[i] + q[i+1]) / 2; for an fp32 x,
+//          x > midpoint  <=>  x > t[i].
+struct Nf4Tables {
+  float q[16];
+  float t[15];
+};
+
+// Derived once per process on the host, from the normal quantiles.
+const Nf4Tables& nf4_tables();
+
+// Process-wide count of kernels launched through the library.
+void count_launches(uint64_t n);
+uint64_t launches_so_far();
+
+// ------------------------------------------------------------------ engine
+// Where the UMMA A operand of the main segment comes from.
+enum AMode : int {
+  A_TMA = 0,     // TMA tile (K- or MN-major per args)
+  A_DEQ_K = 1,   // NF4 dequantised on chip, K-major  (A = W^, rows = n, k along K)
+  A_DEQ_MN = 2,  // NF4 dequantised on chip, MN-major (A = W^T, rows = k, reduction over n)
+};
+
+// Final store of an accumulator element (row, col) of the output tile:
+//   out [row*rs  + col*cs ] = alpha  * v   (fp32 or bf16)
+//   out2[row*rs2 + col*cs2] = alpha2 * v   (bf16, optional)
+struct EpiArgs {
+  void* out;
+  int out_bf16;
+  float alpha;
+  int64_t rs, cs;
+  void* out2;
+  float alpha2;
+  int64_t rs2, cs2;
+};
+
+struct EngineArgs {
+  CUtensorMap tmA;   // main A (A_TMA) or the NF4 code tensor (A_DEQ_*)
+  CUtensorMap tmB;   // main B
+  CUtensorMap tmAx;  // extension A (LoRA term)
+  CUtensorMap tmBx;  // extension B
+  const uint8_t* c2;
+  const float* c1;
+  int64_t wN, wK;    // quantised weight shape (for scale indexing)
+  int rows, cols;    // output extent: UMMA-M side, UMMA-N side
+  int kb_main;       // 64-wide reduction blocks of the main segment
+  int kb_ext;        // 64-wide reduction blocks of the extension (0: none)
+  int splits;        // split of the main reduction across grid.z
+  int a_mn_main, b_mn_main, a_mn_ext, b_mn_ext;
+  float* partial;    // [splits][cols][rows] fp32 when splits > 1
+  EpiArgs epi;
+  int* status;
+  float q[16];
+};
+
+struct GemmPlan {
+  int BN;
+  int m_tiles, n_tiles, splits;
+  size_t partial_bytes;
+};
+
+GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms);
+size_t engine_smem_bytes(int BN, int amode);
+cudaError_t launch_engine(const EngineArgs& a, int amode, const GemmPlan& p, cudaStream_t st);
+cudaError_t launch_split_reduce(const float* partial, int splits, int rows, int cols, const EpiArgs& e,
+                                cudaStream_t st);
+
+// --------------------------------------------------------- quantise kernels
+cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
+                            int* status, cudaStream_t st);
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
+                           uint16_t* out, cudaStream_t st);
+cudaError_t launch_scale_to_bf16(const float* in, int64_t n, float s, uint16_t* out, cudaStream_t st);
+
+}  // namespace qnf4

@@ -1,0 +1,77 @@
+// NF4 codebook and decision thresholds, derived on the host at first use.
+//
+// nlp-lineage "QLoRA" milestone page, section "The idea", NF4 bullet: 16
+// values placed so that each covers an equal share of the normal
+// distribution, with an exact zero.  Construction: 8 positive levels at the
+// standard-normal quantiles of 8 equally spaced probabilities from
+// delta = 1 - (1/32 + 1/30)/2 down towards 1/2, 7 negative levels mirrored
+// from 7 equally spaced probabilities over the same range, plus 0, all
+// divided by the largest level so that the endpoints are exactly -1 and +1.
+//
+// The quantile is computed here by Newton's method on Phi(x) = erfc(-x/sqrt2)/2
+// in extended precision; the result is rounded to fp32.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "internal.h"
+
+namespace qnf4 {
+namespace {
+
+long double phi_cdf(long double x) { return 0.5L * std::erfc(-x / std::sqrt(2.0L)); }
+long double phi_pdf(long double x) {
+  return std::exp(-0.5L * x * x) / std::sqrt(2.0L * 3.14159265358979323846264338327950288L);
+}
+
+long double quantile(long double p) {
+  long double x = 0.0L;
+  for (int it = 0; it < 200; ++it) {
+    const long double step = (phi_cdf(x) - p) / phi_pdf(x);
+    x -= step;
+    if (std::fabs(step) < 1e-19L * (1.0L + std::fabs(x))) break;
+  }
+  return x;
+}
+
+// Largest float <= v.
+float round_down_to_float(double v) {
+  float f = (float)v;
+  if ((double)f > v) f = std::nextafterf(f, -INFINITY);
+  return f;
+}
+
+Nf4Tables build() {
+  const long double delta = 1.0L - 0.5L * (1.0L / 32.0L + 1.0L / 30.0L);
+  long double lv[16];
+  int n = 0;
+  for (int i = 0; i <= 6; ++i) lv[n++] = -quantile(delta + i * (0.5L - delta) / 7.0L);  // negative side
+  lv[n++] = 0.0L;
+  for (int i = 7; i >= 0; --i) lv[n++] = quantile(delta + i * (0.5L - delta) / 8.0L);   // positive side
+  const long double top = lv[15];
+  Nf4Tables t{};
+  for (int i = 0; i < 16; ++i) t.q[i] = (float)(double)(lv[i] / top);
+  t.q[0] = -1.0f;  // lv[0] = -lv[15] exactly by construction
+  t.q[7] = 0.0f;
+  t.q[15] = 1.0f;
+  for (int i = 0; i < 15; ++i) t.t[i] = round_down_to_float(((double)t.q[i] + (double)t.q[i + 1]) * 0.5);
+  return t;
+}
+
+}  // namespace
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+uint64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+
+const Nf4Tables& nf4_tables() {
+  static Nf4Tables tables;
+  static std::once_flag once;
+  std::call_once(once, [] { tables = build(); });
+  return tables;
+}
+
+}  // namespace qnf4

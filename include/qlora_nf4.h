@@ -1,0 +1,174 @@
+/*
+ * qlora_nf4.h -- C ABI of the QLoRA NF4 quantized linear layer for NVIDIA
+ * B200 (sm_100a).  Library: libqlora_nf4.so.
+ *
+ * The operation (nlp-lineage "QLoRA" milestone page, section "The idea",
+ * notation paragraph):
+ *
+ *     Y = X . doubleDequant(c1, c2, W_NF4) + s . X . L1 . L2
+ *
+ * with W frozen in 4 bits and only L1, L2 receiving weight gradients.  The
+ * weight is the nn.Linear weight W[N][K] (out x in); the pages' "X . W" uses
+ * its transpose.  s = alpha / r is the usual LoRA scale (the pages' formula
+ * has s = 1).
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers, owned and allocated by the
+ *     caller.  The library never allocates, frees or synchronises; every call
+ *     is asynchronous on `stream` (a cudaStream_t, 0 = legacy default).
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Tensors are dense row-major.  Every pointer must be 16-byte aligned.
+ *   - Return value: QLORA_OK, or a negative QLORA_ERR_* from the host-side
+ *     checks (nothing is launched then) or from the launch itself.
+ *   - `status_dev` is a device int the kernels write on conditions found on
+ *     the GPU (non-finite weights, an expired internal wait).  Kernels only
+ *     ever store a nonzero QLORA_ERR_* value there; the caller zeroes it and
+ *     reads it after synchronising.  It may be NULL to ignore such reports.
+ *   - Output buffers are overwritten, never accumulated into.
+ *   - Calls that overlap on the GPU must not share a workspace.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+typedef void* qlora_stream_t; /* a cudaStream_t */
+
+enum {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = -1,        /* a required pointer is NULL */
+  QLORA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+  QLORA_ERR_SHAPE = -3,       /* K % 64 != 0, N % 8 != 0, a size < 1 or too large */
+  QLORA_ERR_RANK = -4,        /* r not a multiple of 16 in [16, 128] */
+  QLORA_ERR_WORKSPACE = -5,   /* ws too small (see qlora_workspace_bytes) */
+  QLORA_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
+  QLORA_ERR_NONFINITE = -7,   /* device status: W holds an Inf or NaN */
+  QLORA_ERR_TIMEOUT = -8,     /* device status: an internal wait expired */
+  QLORA_ERR_DEVICE = -9       /* current device is not sm_100 */
+};
+
+/*
+ * The quantized weight (nlp-lineage "QLoRA", section "The idea": blocks of
+ * 64 weights, 4-bit NormalFloat codes, 8-bit block scales c2 and 32-bit
+ * second-level scales c1; inferensys glossary "QLoRA": the scales become
+ * 8-bit floats).
+ *   codes : uint8[N*K/2]   two 4-bit codes per byte, flat row-major order,
+ *                          element 2j in the low nibble, 2j+1 in the high.
+ *   c2    : uint8[N*K/64]  OCP FP8 E4M3 code of each 64-weight block scale.
+ *   c1    : float[ceil(N*K/16384)]  one fp32 scale per 256 consecutive blocks.
+ * Storage: 4 + 8/64 + 32/16384 = 4.127 bits per weight.
+ */
+typedef struct qlora_nf4_weight {
+  uint8_t* codes;
+  uint8_t* c2;
+  float* c1;
+  int64_t n_rows; /* N: output features, >= 1 */
+  int64_t n_cols; /* K: input features, a multiple of 64 */
+} qlora_nf4_weight;
+
+/* Bytes of codes, c2 and c1 for an N x K weight (sizes for the caller's
+ * allocations).  Returns QLORA_ERR_SHAPE for an invalid shape. */
+QLORA_API int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes, size_t* c2_bytes,
+                            size_t* c1_bytes);
+
+/* The 16 NF4 levels the kernels use (ascending, -1 ... 0 ... 1), copied to a
+ * host array.  The library derives them at load from the normal quantiles:
+ * 8 positive and 7 negative levels at equally spaced probabilities between
+ * 1/2 and 1 - (1/32 + 1/30)/2, plus an exact zero, scaled to +-1
+ * (nlp-lineage "QLoRA", section "The idea", NF4 bullet). */
+QLORA_API int qlora_nf4_codebook(float levels[16]);
+
+/*
+ * NF4 double quantisation of a bf16 weight W[N][K] (section "The idea",
+ * NF4 and double-quantisation bullets).
+ *   c_b   = max |w| over each block of 64 (fp32, exact)
+ *   code  = nearest NF4 level to RN32(w / c_b), ties to the lower level
+ *           (all-zero block: code 7, the exact zero)
+ *   c1_g  = RN32(max_{b in g} c_b / 448)      (groups of 256 blocks)
+ *   c2_b  = E4M3_RNE_satfinite(RN32(c_b / c1_g)), 0 when c1_g = 0
+ * W: device bf16[N*K].  out: descriptor whose buffers receive the result
+ * (out->n_rows/n_cols are ignored and N, K used).  A non-finite weight sets
+ * *status_dev = QLORA_ERR_NONFINITE (the outputs are then unspecified).
+ */
+QLORA_API int qlora_nf4_quantize(const uint16_t* W, int64_t N, int64_t K, const qlora_nf4_weight* out,
+                       int* status_dev, qlora_stream_t stream);
+
+/*
+ * doubleDequant(c1, c2, W_NF4) to bf16 (section "The idea", notation
+ * paragraph; inferensys glossary: NF4 dequantised to BFloat16):
+ *   c^_b = RN32(dec_E4M3(c2_b) * c1_g);  w^ = RNbf16(RN32(q[code] * c^_b))
+ * W_out: device bf16[N*K].
+ */
+QLORA_API int qlora_nf4_dequant(const qlora_nf4_weight* w, uint16_t* W_out, int* status_dev,
+                      qlora_stream_t stream);
+
+/* Workspace bytes needed by qlora_linear_fwd and qlora_linear_bwd for M
+ * tokens, an N x K weight and rank r (the maximum over both calls).
+ * Returns 0 for an invalid shape. */
+QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/*
+ * Forward of the quantized linear layer:
+ *   T = X . L1                       (fp32, saved for the backward)
+ *   Y = RNbf16( X . W^T + s . T . L2 )
+ * W^ is the doubleDequant weight, produced tile by tile on chip and never
+ * written to memory (examadda "QLoRA", "The Core Idea": dequantised on the
+ * fly; inferensys: decompressed in shared memory and fed to the tensor cores).
+ *   X   : bf16[M][K]     L1 : bf16[K][r]     L2 : bf16[r][N]
+ *   Y   : bf16[M][N]     T_save : float[M][r]
+ *   ws  : device workspace of ws_bytes >= qlora_workspace_bytes(M, N, K, r)
+ * Requires K % 64 == 0, N % 8 == 0, r % 16 == 0 and 16 <= r <= 128.
+ */
+QLORA_API int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                     const uint16_t* L1, const uint16_t* L2, int r, float s, uint16_t* Y,
+                     float* T_save, void* ws, size_t ws_bytes, int* status_dev,
+                     qlora_stream_t stream);
+
+/*
+ * Backward of the same layer for an upstream gradient dY (gradients flow
+ * through the frozen 4-bit weight into the adapters; W gets none: section
+ * "The idea"; examadda "The Flow"):
+ *   dT  = dY . L2^T
+ *   dX  = RNbf16( dY . W^ + s . dT . L1^T )
+ *   dL1 = s . X^T . dT        (fp32)
+ *   dL2 = s . T^T . dY        (fp32)
+ *   dY : bf16[M][N]   X : bf16[M][K]   T_saved : float[M][r] (from the forward)
+ *   dX : bf16[M][K]   dL1 : float[K][r]   dL2 : float[r][N]
+ * dX, dL1 or dL2 may be NULL to skip that output.  Same shape rules as the
+ * forward.
+ */
+QLORA_API int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const float* T_saved,
+                     const qlora_nf4_weight* w, const uint16_t* L1, const uint16_t* L2, int r,
+                     float s, uint16_t* dX, float* dL1, float* dL2, void* ws, size_t ws_bytes,
+                     int* status_dev, qlora_stream_t stream);
+
+/* Diagnostic timing hook.  When both are non-NULL (cudaEvent_t handles),
+ * the next qlora_linear_fwd / qlora_linear_bwd records `ev_start` on its
+ * stream just before the fused dequant-GEMM launch (Y, resp. dX) and `ev_end`
+ * just after it (and after its split reduction, if any); the hook is then
+ * cleared.  Process-wide, not thread-safe; NULL, NULL clears it. */
+QLORA_API int qlora_set_gemm_events(void* ev_start, void* ev_end);
+
+/* Number of kernels this process has launched through the library so far
+ * (all devices, all calls).  A diagnostic for counting launches. */
+QLORA_API uint64_t qlora_kernel_launches(void);
+
+/* Human-readable text for a QLORA_* code.  Never NULL. */
+QLORA_API const char* qlora_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -30,7 +30,7 @@ __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits", "bf16_bits_to_f64",
     "e4m3_decode", "e4m3_encode", "e4m3_encode_exact",
     "block_absmax", "quantize", "dequant", "decoded_scales",
-    "linear_fwd", "linear_bwd",
+    "linear_fwd", "linear_bwd", "adapter_grads",
     "storage_bytes", "bits_per_weight",
 ]
 
@@ -344,22 +344,31 @@ def linear_fwd(X: np.ndarray, What: np.ndarray, L1: np.ndarray, L2: np.ndarray, 
     return Y, T
 
 
-def linear_bwd(dY, X, What, L1, L2, s, T=None):
-    """Gradients of <Y, dY> for the layer above, fp64.
-
-    dT = dY L2^T; dX = dY W + s dT L1^T; dL2 = s T^T dY; dL1 = s X^T dT.
-    There is no gradient for the frozen weight W.
-    """
+def adapter_grads(dY, X, L1, L2, s, T=None):
+    """The adapters' part of the backward, fp64: dT = dY L2^T,
+    dL2 = s T^T dY, dL1 = s X^T dT.  Returns (dL1, dL2, dT, T)."""
     dY = np.asarray(dY, dtype=np.float64)
     X = np.asarray(X, dtype=np.float64)
     L1 = np.asarray(L1, dtype=np.float64)
     L2 = np.asarray(L2, dtype=np.float64)
     if T is None:
         T = X @ L1
+    T = np.asarray(T, dtype=np.float64)
     dT = dY @ L2.T
-    dX = dY @ np.asarray(What, dtype=np.float64) + s * (dT @ L1.T)
-    dL2 = s * (np.asarray(T, dtype=np.float64).T @ dY)
+    dL2 = s * (T.T @ dY)
     dL1 = s * (X.T @ dT)
+    return dL1, dL2, dT, T
+
+
+def linear_bwd(dY, X, What, L1, L2, s, T=None):
+    """Gradients of <Y, dY> for the layer above, fp64.
+
+    dT = dY L2^T; dX = dY W + s dT L1^T; dL2 = s T^T dY; dL1 = s X^T dT.
+    There is no gradient for the frozen weight W.
+    """
+    dL1, dL2, dT, _ = adapter_grads(dY, X, L1, L2, s, T)
+    dY = np.asarray(dY, dtype=np.float64)
+    dX = dY @ np.asarray(What, dtype=np.float64) + s * (dT @ np.asarray(L1, dtype=np.float64).T)
     return dX, dL1, dL2, dT
 
 

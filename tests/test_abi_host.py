@@ -1,0 +1,95 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every symbol the header declares, derives the same NF4 codebook as the
+oracle on its own, and rejects bad arguments before touching a device."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_15_b200 as q
+    from bit_nf4_quantized_15_b200 import build
+    build.build()
+    return q
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(qlora_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    syms = declared_symbols()
+    for name in ("qlora_nf4_quantize", "qlora_nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(q):
+    h = ctypes.CDLL(q.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(h, name), name
+
+
+def test_codebook_matches_oracle_bitwise(q):
+    ours = np.array(q.codebook(), dtype=np.float32)
+    ref = O.nf4_codebook()
+    assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32))
+
+
+def test_storage_bytes(q):
+    nc, n2, n1 = q.storage_bytes(4096, 4096)
+    assert (nc, n2, n1) == (4096 * 4096 // 2, 4096 * 4096 // 64, 4 * (4096 * 4096 // 16384))
+    assert (nc + n2 + n1) * 8 / (4096 * 4096) == O.bits_per_weight(4096, 4096)
+    assert (nc + n2 + n1) == O.storage_bytes(4096, 4096)
+    nc, n2, n1 = q.storage_bytes(5, 64 * 300)            # partial last c1 group
+    assert n1 == 4 * 6
+    with pytest.raises(q.QLoRAError):
+        q.storage_bytes(4, 100)
+
+
+def test_status_strings(q):
+    for code in range(-9, 1):
+        assert q.status_string(code)
+    assert "unknown" in q.status_string(-99)
+
+
+def test_workspace_bytes_host(q):
+    L = q.lib()
+    assert L.qlora_workspace_bytes(16, 4096, 4096, 16) > 0
+    assert L.qlora_workspace_bytes(16, 4096, 4096, 17) == 0      # bad rank
+    assert L.qlora_workspace_bytes(16, 4096, 100, 16) == 0       # K % 64
+    assert L.qlora_workspace_bytes(16, 4100, 4096, 16) == 0      # N % 8
+
+
+def test_argument_checks_before_any_launch(q):
+    """Bad arguments are rejected on the host: these fake, never dereferenced
+    pointers would fault if any kernel were launched."""
+    L = q.lib()
+    P = ctypes.c_void_p
+    w = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 128)
+    fake = P(0x10000)
+    # NULL input
+    assert L.qlora_linear_fwd(None, 4, ctypes.byref(w), fake, fake, 16, 1.0, fake, fake, fake, 1 << 20, None, None) == -1
+    # rank
+    assert L.qlora_linear_fwd(fake, 4, ctypes.byref(w), fake, fake, 17, 1.0, fake, fake, fake, 1 << 20, None, None) == -4
+    # shape: K % 64
+    w_bad = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 100)
+    assert L.qlora_linear_fwd(fake, 4, ctypes.byref(w_bad), fake, fake, 16, 1.0, fake, fake, fake, 1 << 20, None, None) == -3
+    # alignment
+    assert L.qlora_linear_fwd(P(0x10008), 4, ctypes.byref(w), fake, fake, 16, 1.0, fake, fake, fake, 1 << 20, None, None) == -2
+    assert L.qlora_linear_bwd(fake, fake, 4, fake, ctypes.byref(w), fake, fake, 16, 1.0, P(0x10004), None, None,
+                              fake, 1 << 20, None, None) == -2
+    # quantize
+    assert L.qlora_nf4_quantize(fake, 64, 100, ctypes.byref(w), None, None) == -3
+    assert L.qlora_nf4_quantize(None, 64, 128, ctypes.byref(w), None, None) == -1
+    assert L.qlora_nf4_dequant(ctypes.byref(w_bad), fake, None, None) == -3
