@@ -407,6 +407,27 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_profile_case(args):
+    """One linear (gate, 11008x4096, 4096 tokens, r = 64): quantise, then two
+    forward + backward passes; the second is the one to capture with ncu
+    (engine launches in order: T, Y, dT, dX, dL1, dL2)."""
+    import torch
+    import bit_nf4_quantized_15_b200 as q
+    from bit_nf4_quantized_15_b200 import workloads as WL
+    wl = WL.WORKLOADS[WORKLOAD]
+    lin = wl.linears[4]
+    t = WL.make_linear(wl, lin, seed=4, device="cuda")
+    w = q.quantize(t["W"])
+    ws = torch.empty(q.workspace_bytes(wl.M, lin.N, lin.K, wl.r), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        Y, T = q.linear_fwd(t["X"], w, t["L1"], t["L2"], wl.s, ws=ws)
+        q.linear_bwd(t["dY"], t["X"], T, w, t["L1"], t["L2"], wl.s, ws=ws)
+    torch.cuda.synchronize()
+    assert q.read_status() == 0
+    print(json.dumps({"profile_case": f"{lin.name} {lin.N}x{lin.K}", "tokens": wl.M, "r": wl.r,
+                      "launches": q.kernel_launches()}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,8 +436,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true", help="run the single-linear ncu capture case")
     args = ap.parse_args(argv)
-    if args.impl == "reference":
+    if args.profile:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -28,14 +28,15 @@ QDEV uint4 ld_stream_v4(const void* p) {
 // x = RN32(w / c) for |w| <= c.  For c in [2^-90, 2^100) a correctly rounded
 // reciprocal, one product and one fused correction step give the IEEE
 // quotient's NF4 code for every bf16 pair (checked exhaustively); other
-// scales use the IEEE division directly.
+// finite scales use the IEEE division directly.  A zero or non-finite scale
+// gives x = 0 (a non-finite block is reported through the status word).
 QDEV float ratio(float w, float c, float rc, bool fast) {
   if (fast) {
     const float q0 = __fmul_rn(w, rc);
     const float e = __fmaf_rn(-q0, c, w);
     return __fmaf_rn(e, rc, q0);
   }
-  return c > 0.0f ? __fdiv_rn(w, c) : 0.0f;
+  return (c > 0.0f && c <= 3.402823466e38f) ? __fdiv_rn(w, c) : 0.0f;
 }
 
 // Code of x via a 129-entry bucket table: bucket j = RN(64 x) + 64 covers the
@@ -45,7 +46,7 @@ QDEV float ratio(float w, float c, float rc, bool fast) {
 QDEV uint32_t nf4_code(float x, const float2* bucket) {
   const float y = __fmaf_rn(x, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64
   const int j = __float_as_int(y) - 0x4B400000;       // bits of 1.5 * 2^23
-  const float2 b = bucket[j];
+  const float2 b = bucket[min((unsigned)j, 128u)];     // |x| <= 1 keeps j in [0, 128]
   return (uint32_t)__float_as_int(b.y) + (x > b.x ? 1u : 0u);
 }
 
