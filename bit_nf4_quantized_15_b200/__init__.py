@@ -59,6 +59,8 @@ _SIGS = {
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_kernel_launches": (ctypes.c_uint64, []),
     "qlora_set_gemm_events": (ctypes.c_int, [_P, _P]),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P, ctypes.c_int,
+                                                ctypes.c_float, _P, _P, _P, _P]),
 }
 
 

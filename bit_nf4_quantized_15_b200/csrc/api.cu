@@ -179,6 +179,7 @@ const char* qlora_status_string(int code) {
     case QLORA_ERR_NONFINITE: return "weight holds an Inf or NaN";
     case QLORA_ERR_TIMEOUT: return "an internal GPU wait expired";
     case QLORA_ERR_DEVICE: return "current device is not an sm_100 GPU";
+    case QLORA_ERR_SCRATCH_LIMIT: return "problem needs more workspace than the library's 8 MiB static scratch";
   }
   return "unknown status";
 }

@@ -55,7 +55,8 @@ enum {
   QLORA_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
   QLORA_ERR_NONFINITE = -7,   /* device status: W holds an Inf or NaN */
   QLORA_ERR_TIMEOUT = -8,     /* device status: an internal wait expired */
-  QLORA_ERR_DEVICE = -9       /* current device is not sm_100 */
+  QLORA_ERR_DEVICE = -9,      /* current device is not sm_100 */
+  QLORA_ERR_SCRATCH_LIMIT = -10 /* problem needs more than the library's static scratch */
 };
 
 /*
@@ -152,6 +153,27 @@ QLORA_API int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M,
                      const qlora_nf4_weight* w, const uint16_t* L1, const uint16_t* L2, int r,
                      float s, uint16_t* dX, float* dL1, float* dL2, void* ws, size_t ws_bytes,
                      int* status_dev, qlora_stream_t stream);
+
+/*
+ * Forward without a caller workspace, for callers that cannot allocate
+ * device memory (no counterpart on the pages: this is an interface for
+ * embedding the layer, not part of the method).  Such callers include
+ * plugins and custom operators run by a host framework that owns the device
+ * memory pool and forbids allocation inside its execute callback, and
+ * serving loops whose policy forbids cudaMalloc after start-up.  Same
+ * arguments and results as qlora_linear_fwd minus ws / ws_bytes: the
+ * workspace is a static device array inside the library, 8 MiB on every GPU
+ * that loads it, held until exit.  A problem whose qlora_workspace_bytes()
+ * exceeds 8 MiB is rejected with QLORA_ERR_SCRATCH_LIMIT before anything is
+ * launched.  The first call on a device looks up the array's device address
+ * (once per device, that device current); make that first call before any
+ * stream capture.  All calls share the one array: calls that overlap on the
+ * GPU race and must be serialised by the caller.  Allocates nothing.
+ */
+QLORA_API int qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                                       const uint16_t* L1, const uint16_t* L2, int r, float s,
+                                       uint16_t* Y, float* T_save, int* status_dev,
+                                       qlora_stream_t stream);
 
 /* Diagnostic timing hook.  When both are non-NULL (cudaEvent_t handles),
  * the next qlora_linear_fwd / qlora_linear_bwd records `ev_start` on its

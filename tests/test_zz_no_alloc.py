@@ -1,0 +1,76 @@
+"""The forward entry point that allocates nothing (qlora_linear_fwd_noalloc).
+
+It exists for callers that cannot allocate device memory themselves, such as
+operators run inside a host framework that owns the device memory pool and
+forbids allocation while it executes them, or serving loops that must not
+call cudaMalloc after start-up.  Instead of a caller workspace it uses a
+static 8 MiB device array inside the library.  Checked here through the C ABI
+against the regular forward (with a caller workspace), within the parity
+tolerance, on two calls in a row (the array keeps the previous call's
+contents), and for its size limit.  This file sorts last so a run that stops
+at the first failure has run everything else before it.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import assert_close, from_bits, to_f64
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_LIMIT = -10
+
+
+def _bf(rng, shape, std):
+    x = torch.from_numpy(rng.normal(0, std, shape).astype(np.float32))
+    return x.to(torch.bfloat16).cuda()
+
+
+def _noalloc(q, X, w, L1, L2, s, Y, T, status):
+    d = w.descriptor()
+    M, r = X.shape[0], L1.shape[1]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return q.lib().qlora_linear_fwd_noalloc(ctypes.c_void_p(X.data_ptr()), M, ctypes.byref(d),
+                                            ctypes.c_void_p(L1.data_ptr()), ctypes.c_void_p(L2.data_ptr()), r,
+                                            float(s), ctypes.c_void_p(Y.data_ptr()), ctypes.c_void_p(T.data_ptr()),
+                                            ctypes.c_void_p(status.data_ptr()), stream)
+
+
+@pytest.mark.parametrize("M,N,K,r", [(16, 4096, 4096, 16), (200, 384, 512, 64), (37, 136, 256, 32)])
+def test_noalloc_forward_matches_regular_forward(lib, M, N, K, r):
+    rng = np.random.default_rng(M + N + K + r)
+    X, W = _bf(rng, (M, K), 1.0), _bf(rng, (N, K), 0.02)
+    L1, L2 = _bf(rng, (K, r), K ** -0.5), _bf(rng, (r, N), 0.05)
+    s = 16.0 / r
+    assert lib.workspace_bytes(M, N, K, r) <= 8 << 20
+    w = lib.quantize(W)
+    Y_ref, T_ref = lib.linear_fwd(X, w, L1, L2, s)
+    torch.cuda.synchronize()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        T = torch.full((M, r), float("nan"), dtype=torch.float32, device="cuda")
+        assert _noalloc(lib, X, w, L1, L2, s, Y, T, status) == 0
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert_close(to_f64(Y), to_f64(Y_ref), "Y")
+        assert_close(to_f64(T), to_f64(T_ref), "T")
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(lib):
+    M, N, K, r = 65536, 8, 64, 128          # s.T alone is 16 MiB of workspace
+    assert lib.workspace_bytes(M, N, K, r) > 8 << 20
+    rng = np.random.default_rng(1)
+    X, W = _bf(rng, (M, K), 1.0), _bf(rng, (N, K), 0.02)
+    L1, L2 = _bf(rng, (K, r), 0.1), _bf(rng, (r, N), 0.1)
+    w = lib.quantize(W)
+    Y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.zeros((M, r), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert _noalloc(lib, X, w, L1, L2, 1.0, Y, T, status) == SCRATCH_LIMIT
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(Y).item() == 0 and torch.count_nonzero(T).item() == 0
+    assert "8 MiB" in lib.status_string(SCRATCH_LIMIT)
