@@ -80,11 +80,12 @@ int map_operand(CUtensorMap* m, const void* base, int mn_major, uint64_t mn_exte
 
 int map_codes(CUtensorMap* m, const uint8_t* codes, int64_t N, int64_t K, int mn_mode) {
   // codes viewed as uint8 [N][K/2]
+  // Swizzled so that the dequant threads' 16-byte reads are bank-conflict free.
   if (!mn_mode)
     return make_map(m, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 32, 128,
-                    CU_TENSOR_MAP_SWIZZLE_NONE);
+                    CU_TENSOR_MAP_SWIZZLE_32B);
   return make_map(m, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 64, 64,
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
+                  CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -127,6 +127,16 @@ QDEV void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t id
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same with A read from tensor memory (M = 128 lanes, 8 columns per K = 16:
+// column j of a lane holds the two bf16 elements 2j (low half) and 2j+1).
+QDEV void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on `bar` when every previously issued tcgen05.mma has finished.
 QDEV void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -145,6 +155,16 @@ QDEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 QDEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 32 lanes x 16 consecutive 32-bit columns, registers -> tensor memory.
+QDEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+QDEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled canonical layout.
 //   K-major : atoms of 8 rows x 128 B; sbo = byte stride between 8-row groups.
@@ -186,6 +206,45 @@ QDEV float decode_scale(uint32_t c2code, float c1v) { return __fmul_rn(e4m3_to_f
 QDEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------- NF4 block table in registers
+// For one 64-weight block with decoded scale c^, the 16 possible dequantised
+// values T[i] = RNbf16(RN32(q[i] * c^)) are computed once and kept as byte
+// planes: L[m] holds the low bytes of T[4m .. 4m+3], H[m] the high bytes.
+struct Nf4BlockTable {
+  uint32_t L[4], H[4];
+};
+
+QDEV Nf4BlockTable nf4_block_table(const float (&q)[16], float chat) {
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) P[j] = pack_bf16x2(__fmul_rn(q[2 * j], chat), __fmul_rn(q[2 * j + 1], chat));
+  Nf4BlockTable t;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    t.L[m] = __byte_perm(P[2 * m], P[2 * m + 1], 0x6420);
+    t.H[m] = __byte_perm(P[2 * m], P[2 * m + 1], 0x7531);
+  }
+  return t;
+}
+
+// Four codes (nibbles 0..3 of h) -> two bf16x2 words (T[c0] | T[c1] << 16,
+// T[c2] | T[c3] << 16) by byte permutes: the low three bits of each code pick
+// a byte out of an 8-entry plane pair, bit 3 picks the plane pair.
+QDEV void nf4_lookup4(uint32_t h, const Nf4BlockTable& t, uint32_t& out0, uint32_t& out1) {
+  const uint32_t sel = h & 0x7777u;
+  const uint32_t hi8 = ((h >> 1) & 0x4444u) | 0x3210u;
+  const uint32_t lo = __byte_perm(__byte_perm(t.L[0], t.L[1], sel), __byte_perm(t.L[2], t.L[3], sel), hi8);
+  const uint32_t hi = __byte_perm(__byte_perm(t.H[0], t.H[1], sel), __byte_perm(t.H[2], t.H[3], sel), hi8);
+  out0 = __byte_perm(lo, hi, 0x5140);
+  out1 = __byte_perm(lo, hi, 0x7362);
+}
+
+// Eight codes (one 32-bit word, element i in nibble i) -> four bf16x2 words.
+QDEV void nf4_lookup8(uint32_t w, const Nf4BlockTable& t, uint32_t* out) {
+  nf4_lookup4(w, t, out[0], out[1]);
+  nf4_lookup4(w >> 16, t, out[2], out[3]);
 }
 
 }  // namespace qnf4

@@ -26,12 +26,19 @@ namespace qnf4 {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
-constexpr int kA = 16384;  // 128 rows x 64 bf16
+constexpr int kDeqWarps = 8;                   // warps 2..9: dequant, then epilogue
+constexpr int kThreads = 64 + 32 * kDeqWarps;  // + producer warp + UMMA warp
+constexpr int kA = 16384;                      // 128 rows x 64 bf16
 
-template <int BN>
+// Tensor-memory columns: the fp32 accumulator (BN columns, at least 32) and,
+// for the forward fused GEMM, the dequantised A tile of every stage
+// (128 lanes x 32 columns: 64 bf16 per lane).
+template <int BN, int AMODE>
 struct Tmem {
-  static constexpr uint32_t cols = BN < 32 ? 32 : BN;
+  static constexpr uint32_t acc = BN < 32 ? 32 : BN;
+  static constexpr uint32_t a_col = acc;
+  static constexpr uint32_t need = acc + (AMODE == A_DEQ_K ? kStages * 32 : 0);
+  static constexpr uint32_t cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 };
 
 template <int BN, int AMODE>
@@ -74,9 +81,20 @@ QDEV void epi_store(const EpiArgs& e, int64_t row, int64_t col, float v) {
   }
 }
 
+// Warp-wide wait: lane 0 polls (bounded), then every lane takes one
+// acquiring look at the completed phase.
+QDEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status, int lane) {
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (ok) mbar_try_wait(smem_u32(bar), parity);
+  return ok != 0;
+}
+
 template <int BN, int AMODE>
 __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_constant__ EngineArgs args) {
   using L = Layout<BN, AMODE>;
+  using TM = Tmem<BN, AMODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -85,7 +103,6 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
   uint64_t* accum = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* lut = reinterpret_cast<float*>(tmem_slot + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = blockIdx.x * 128, col0 = blockIdx.y * BN, z = blockIdx.z;
@@ -97,14 +114,13 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(afull + s, 4);
+      mbar_init(afull + s, kDeqWarps);
       mbar_init(empty + s, 1);
     }
     mbar_init(accum, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (tid < 16) lut[tid] = args.q[tid];
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&args.tmA);
     tma_prefetch_desc(&args.tmB);
@@ -114,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Tmem<BN>::cols);
+    tmem_alloc(tmem_slot, TM::cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -156,23 +172,31 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
       const int a_mn_main = AMODE == A_DEQ_MN ? 1 : (AMODE == A_DEQ_K ? 0 : args.a_mn_main);
       const uint32_t id_main = idesc_bf16(128, BN, a_mn_main, args.b_mn_main);
       const uint32_t id_ext = idesc_bf16(128, BN, args.a_mn_ext, args.b_mn_ext);
-      bool ok = true;
-      for (int it = 0; it < n_iters && ok; ++it) {
+      for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const bool ext = it >= my_kb;
-        ok = mbar_wait(full + s, ph, abort_flag, args.status);
+        bool ok = mbar_wait(full + s, ph, abort_flag, args.status);
         if (ok && AMODE != A_TMA && !ext) ok = mbar_wait(afull + s, ph, abort_flag, args.status);
         if (!ok) break;
         tc_fence_after();
         const uint8_t* sa = smem + s * L::STAGE;
         const uint8_t* sb = sa + kA;
-        const int amn = ext ? args.a_mn_ext : a_mn_main;
-        const int bmn = ext ? args.b_mn_ext : args.b_mn_main;
-        const uint32_t id = ext ? id_ext : id_main;
+        if (AMODE == A_DEQ_K && !ext) {
+          // A: dequantised weight tile in tensor memory, 8 columns per K = 16
+          const uint32_t a_tmem = tmem_d + TM::a_col + (uint32_t)(s * 32);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem_d, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (it | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_tmem_a(tmem_d, a_tmem + kk * 8, operand_desc(sb, args.b_mn_main, kk), id_main,
+                             (it | kk) != 0);
+        } else {
+          const int amn = ext ? args.a_mn_ext : a_mn_main;
+          const int bmn = ext ? args.b_mn_ext : args.b_mn_main;
+          const uint32_t id = ext ? id_ext : id_main;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_d, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (it | kk) != 0);
+        }
         umma_commit(empty + s);
       }
       umma_commit(accum);
@@ -180,13 +204,22 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
     }
     __syncwarp();
   } else {
-    const int e = tid - 64;  // 0..127
+    const int dw = warp - 2;     // dequant warp 0..7
+    const int q4 = warp & 3;     // TMEM lane quarter this warp may access
+    const int64_t bpr = args.wK / 64;  // NF4 blocks per weight row
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = args.q[i];
     // ------------------------------------------------------------- dequant
     if (AMODE == A_DEQ_K) {
-      // Thread e owns output row n = row0 + e (one NF4 block of 64 per stage).
-      const int64_t n = row0 + e;
+      // Row rl of the tile = TMEM lane; this warp covers k = 32*half .. +31 of
+      // each 64-wide stage (one half of the row's NF4 block).
+      const int half = dw >> 2;
+      const int rl = q4 * 32 + lane;
+      const int64_t n = row0 + rl;
       const bool valid = n < args.wN;
-      const int64_t bpr = args.wK / 64;  // blocks per weight row
+      const uint32_t taddr = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col + (uint32_t)(half * 16);
+      const int cofs = rl * 32 + ((half ^ ((rl >> 2) & 1)) << 4);  // 32-byte-swizzled code tile
       uint32_t c2raw = 0;
       float c1v = 0.0f;
       if (valid && my_kb > 0) {
@@ -194,94 +227,81 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
         c2raw = __ldg(args.c2 + f);
         c1v = __ldg(args.c1 + (f >> 8));
       }
-      const uint32_t swz = (uint32_t)(e & 7);
       for (int it = 0; it < my_kb; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
-        if (valid && it + 1 < my_kb) {  // prefetch the next stage's scale
+        if (valid && it + 1 < my_kb) {  // the next stage's scale, one stage ahead
           const int64_t f = n * bpr + kb_lo + it + 1;
           c2raw = __ldg(args.c2 + f);
           c1v = __ldg(args.c1 + (f >> 8));
         }
-        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
-        if (!mbar_wait(full + s, ph, abort_flag, args.status)) break;
-        const uint8_t* sc = smem + s * L::STAGE + kA + L::B;
-        uint8_t* sa = smem + s * L::STAGE;
-        const uint4 cw0 = *reinterpret_cast<const uint4*>(sc + e * 32);
-        const uint4 cw1 = *reinterpret_cast<const uint4*>(sc + e * 32 + 16);
-        const uint32_t words[8] = {cw0.x, cw0.y, cw0.z, cw0.w, cw1.x, cw1.y, cw1.z, cw1.w};
-        uint8_t* rowp = sa + (e >> 3) * 1024 + (e & 7) * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {  // chunk c: k = 8c .. 8c+7
-          const uint32_t w = words[c];
-          uint32_t o[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t b = w >> (8 * k);
-            o[k] = pack_bf16x2(__fmul_rn(lut[b & 15u], chat), __fmul_rn(lut[(b >> 4) & 15u], chat));
-          }
-          *reinterpret_cast<uint4*>(rowp + (((uint32_t)c ^ swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        fence_proxy_async_smem();
+        const Nf4BlockTable tab = nf4_block_table(q, chat);
+        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane)) break;
+        tc_fence_after();
+        if (!warp_wait(full + s, ph, abort_flag, args.status, lane)) break;
+        const uint4 cw = *reinterpret_cast<const uint4*>(smem + s * L::STAGE + kA + L::B + cofs);
+        uint32_t o[16];
+        nf4_lookup8(cw.x, tab, o + 0);
+        nf4_lookup8(cw.y, tab, o + 4);
+        nf4_lookup8(cw.z, tab, o + 8);
+        nf4_lookup8(cw.w, tab, o + 12);
+        tmem_st16(taddr + (uint32_t)(s * 32), o);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(afull + s);
       }
     } else if (AMODE == A_DEQ_MN) {
-      // A = W^T: rows are k (W columns), the reduction runs over n (W rows).
-      // Thread e: 16 consecutive k (w2 = e % 8 -> k_local = 16 w2) of rows
-      // n_local = e/8 + 16 i, i = 0..3.
-      const int w2 = e & 7, rg = e >> 3;
-      const int64_t bpr = args.wK / 64;
-      const int64_t kblk = (int64_t)(row0 >> 6) + (w2 >> 2);
+      // A = W^T in shared memory, MN-major: rows are k (W columns), the
+      // reduction runs over n (W rows).  Thread (u, half): W row n0 + nl,
+      // 32 consecutive k (k_local = 64*mb + 32*half ..) of one NF4 block.
+      const int e = tid - 64;
+      const int u = e & 127, half = e >> 7;
+      const int nl = u & 63, mb = u >> 6;
+      const int64_t kblk = (int64_t)(row0 >> 6) + mb;
       const bool kvalid = kblk < bpr;
-      const int mb = w2 >> 2;
-      const uint32_t cA = (uint32_t)(2 * (w2 & 3));
-      const bool swap = w2 >= 4;  // store order that keeps an 8-thread phase conflict-free
+      const int r8 = nl & 7;
+      const int cofs = nl * 64 + (((2 * mb + half) ^ ((nl >> 1) & 3)) << 4);  // 64-byte-swizzled code tile
+      const int aofs = mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
+      uint32_t c2raw = 0;
+      float c1v = 0.0f;
+      {
+        const int64_t nn = (int64_t)kb_lo * 64 + nl;
+        if (kvalid && nn < args.wN && my_kb > 0) {
+          const int64_t f = nn * bpr + kblk;
+          c2raw = __ldg(args.c2 + f);
+          c1v = __ldg(args.c1 + (f >> 8));
+        }
+      }
       for (int it = 0; it < my_kb; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        const int64_t n0 = (int64_t)(kb_lo + it) * 64;
-        uint32_t c2r[4];
-        float c1r[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int64_t n = n0 + rg + 16 * i;
-          c2r[i] = 0;
-          c1r[i] = 0.0f;
-          if (kvalid && n < args.wN) {
-            const int64_t f = n * bpr + kblk;
-            c2r[i] = __ldg(args.c2 + f);
-            c1r[i] = __ldg(args.c1 + (f >> 8));
+        const int64_t nn = (int64_t)(kb_lo + it) * 64 + nl;
+        const bool valid = kvalid && nn < args.wN;
+        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        if (it + 1 < my_kb) {
+          const int64_t nx = nn + 64;
+          c2raw = 0;
+          c1v = 0.0f;
+          if (kvalid && nx < args.wN) {
+            const int64_t f = nx * bpr + kblk;
+            c2raw = __ldg(args.c2 + f);
+            c1v = __ldg(args.c1 + (f >> 8));
           }
         }
-        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
-        if (!mbar_wait(full + s, ph, abort_flag, args.status)) break;
-        const uint8_t* sc = smem + s * L::STAGE + kA + L::B;
+        const Nf4BlockTable tab = nf4_block_table(q, chat);
+        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane)) break;
+        if (!warp_wait(full + s, ph, abort_flag, args.status, lane)) break;
         uint8_t* sa = smem + s * L::STAGE;
+        const uint4 cw = *reinterpret_cast<const uint4*>(sa + kA + L::B + cofs);
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int nl = rg + 16 * i;
-          const float chat = (c1r[i] != 0.0f) ? decode_scale(c2r[i], c1r[i]) : 0.0f;
-          const uint2 cw = *reinterpret_cast<const uint2*>(sc + nl * 64 + w2 * 8);
-          uint32_t o[8];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t b0 = cw.x >> (8 * k), b1 = cw.y >> (8 * k);
-            o[k] = pack_bf16x2(__fmul_rn(lut[b0 & 15u], chat), __fmul_rn(lut[(b0 >> 4) & 15u], chat));
-            o[4 + k] = pack_bf16x2(__fmul_rn(lut[b1 & 15u], chat), __fmul_rn(lut[(b1 >> 4) & 15u], chat));
-          }
-          const uint32_t r8 = (uint32_t)(nl & 7);
-          uint8_t* atom = sa + mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
-          const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]);
-          const uint4 hi = make_uint4(o[4], o[5], o[6], o[7]);
-          if (!swap) {
-            *reinterpret_cast<uint4*>(atom + ((cA ^ r8) << 4)) = lo;
-            *reinterpret_cast<uint4*>(atom + (((cA + 1) ^ r8) << 4)) = hi;
-          } else {
-            *reinterpret_cast<uint4*>(atom + (((cA + 1) ^ r8) << 4)) = hi;
-            *reinterpret_cast<uint4*>(atom + ((cA ^ r8) << 4)) = lo;
-          }
+        for (int j = 0; j < 4; ++j) {
+          uint32_t o[4];
+          nf4_lookup8(words[j], tab, o);
+          const uint32_t c = (uint32_t)(4 * half + j);
+          *reinterpret_cast<uint4*>(sa + aofs + ((c ^ (uint32_t)r8) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -289,11 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
       }
     }
     // ------------------------------------------------------------ epilogue
-    const bool ok = mbar_wait(accum, 0, abort_flag, args.status);
+    // Two warps per lane quarter: warp group g stores columns [g*BN/2, ...).
+    const bool ok = warp_wait(accum, 0, abort_flag, args.status, lane);
     tc_fence_after();
-    const int q4 = warp & 3;
+    const int g = dw >> 2;
+    const int c_lo = BN >= 32 ? g * (BN / 2) : 0;
+    const int c_hi = BN >= 32 ? c_lo + BN / 2 : (g == 0 ? BN : 0);
     const int64_t row = row0 + q4 * 32 + lane;
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = c_lo; c < c_hi; c += 16) {
       uint32_t v[16];
       tmem_ld16(tmem_d + ((uint32_t)(q4 * 32) << 16) + (uint32_t)c, v);
       tmem_wait_ld();
@@ -315,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
     if (*abort_flag && lane == 0 && committed_accum) mbar_wait_drain(accum, 0, 10000000ull);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_d, Tmem<BN>::cols);
+    tmem_dealloc(tmem_d, TM::cols);
   }
 }
 
