@@ -410,7 +410,8 @@ def run_ours(args):
 def run_profile_case(args):
     """One linear (gate, 11008x4096, 4096 tokens, r = 64): quantise, then two
     forward + backward passes; the second is the one to capture with ncu
-    (engine launches in order: T, Y, dT, dX, dL1, dL2)."""
+    (engine launches in order: T, Y, dT, dX, dL1, dL2).  Then two quantise and
+    two dequantise passes of a 32768x4096 weight."""
     import torch
     import bit_nf4_quantized_15_b200 as q
     from bit_nf4_quantized_15_b200 import workloads as WL
@@ -422,6 +423,14 @@ def run_profile_case(args):
     for _ in range(2):
         Y, T = q.linear_fwd(t["X"], w, t["L1"], t["L2"], wl.s, ws=ws)
         q.linear_bwd(t["dY"], t["X"], T, w, t["L1"], t["L2"], wl.s, ws=ws)
+    # then two NF4 quantise and two dequantise passes over a 256 MB bf16 weight (> L2)
+    Wbig = torch.randn((32768, 4096), device="cuda", dtype=torch.float32).mul_(0.02).to(torch.bfloat16)
+    wbig = q.NF4Weight.empty(32768, 4096, "cuda")
+    out = torch.empty_like(Wbig)
+    for _ in range(2):
+        q.quantize_into(Wbig, wbig)
+    for _ in range(2):
+        q.dequant(wbig, out=out)
     torch.cuda.synchronize()
     assert q.read_status() == 0
     print(json.dumps({"profile_case": f"{lin.name} {lin.N}x{lin.K}", "tokens": wl.M, "r": wl.r,

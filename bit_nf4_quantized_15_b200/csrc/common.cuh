@@ -60,6 +60,21 @@ QDEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the thread may be suspended in hardware (up to about a
+// millisecond) until the phase completes instead of returning at once, so a
+// waiting warp does not take issue slots from the warps doing work.
+QDEV bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Bounded: returns
 // false (after flagging the CTA and the caller's status) on timeout or when
 // another role of the CTA has already aborted.
@@ -67,15 +82,13 @@ QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, in
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > QNF4_WAIT_NS) {
-        *abort_flag = 1;
-        report(status, QLORA_ERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > QNF4_WAIT_NS) {
+      *abort_flag = 1;
+      report(status, QLORA_ERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -229,12 +242,12 @@ QDEV Nf4BlockTable nf4_block_table(const float (&q)[16], float chat) {
   return t;
 }
 
-// Four codes (nibbles 0..3 of h) -> two bf16x2 words (T[c0] | T[c1] << 16,
-// T[c2] | T[c3] << 16) by byte permutes: the low three bits of each code pick
-// a byte out of an 8-entry plane pair, bit 3 picks the plane pair.
-QDEV void nf4_lookup4(uint32_t h, const Nf4BlockTable& t, uint32_t& out0, uint32_t& out1) {
-  const uint32_t sel = h & 0x7777u;
-  const uint32_t hi8 = ((h >> 1) & 0x4444u) | 0x3210u;
+// Four codes -> two bf16x2 words (T[c0] | T[c1] << 16, T[c2] | T[c3] << 16)
+// by byte permutes: `sel` holds the codes' low three bits (one per nibble),
+// they pick a byte out of an 8-entry plane pair; `hi8` (nibble i = i + 4 when
+// code i >= 8) picks the plane pair.  A byte permute reads only the low 16
+// bits of its selector.
+QDEV void nf4_lookup4(uint32_t sel, uint32_t hi8, const Nf4BlockTable& t, uint32_t& out0, uint32_t& out1) {
   const uint32_t lo = __byte_perm(__byte_perm(t.L[0], t.L[1], sel), __byte_perm(t.L[2], t.L[3], sel), hi8);
   const uint32_t hi = __byte_perm(__byte_perm(t.H[0], t.H[1], sel), __byte_perm(t.H[2], t.H[3], sel), hi8);
   out0 = __byte_perm(lo, hi, 0x5140);
@@ -243,8 +256,10 @@ QDEV void nf4_lookup4(uint32_t h, const Nf4BlockTable& t, uint32_t& out0, uint32
 
 // Eight codes (one 32-bit word, element i in nibble i) -> four bf16x2 words.
 QDEV void nf4_lookup8(uint32_t w, const Nf4BlockTable& t, uint32_t* out) {
-  nf4_lookup4(w, t, out[0], out[1]);
-  nf4_lookup4(w >> 16, t, out[2], out[3]);
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t hi8 = ((w >> 1) & 0x44444444u) | 0x32103210u;
+  nf4_lookup4(sel, hi8, t, out[0], out[1]);
+  nf4_lookup4(sel >> 16, hi8 >> 16, t, out[2], out[3]);
 }
 
 }  // namespace qnf4

@@ -26,7 +26,8 @@ namespace qnf4 {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kDeqWarps = 8;                   // warps 2..9: dequant, then epilogue
+constexpr int kDeqWarps = 16;                  // warps 2..17: dequant, then epilogue
+constexpr int kGroupWarps = 4;                 // one group of 4 warps per ring stage
 constexpr int kThreads = 64 + 32 * kDeqWarps;  // + producer warp + UMMA warp
 constexpr int kA = 16384;                      // 128 rows x 64 bf16
 
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(afull + s, kDeqWarps);
+      mbar_init(afull + s, kGroupWarps);
       mbar_init(empty + s, 1);
     }
     mbar_init(accum, 1);
@@ -204,84 +205,92 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
     }
     __syncwarp();
   } else {
-    const int dw = warp - 2;     // dequant warp 0..7
-    const int q4 = warp & 3;     // TMEM lane quarter this warp may access
+    const int dw = warp - 2;           // dequant warp 0..15
+    const int q4 = warp & 3;           // TMEM lane quarter this warp may access
+    const int grp = dw >> 2;           // group = the ring stage these 4 warps fill
     const int64_t bpr = args.wK / 64;  // NF4 blocks per weight row
     float q[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) q[i] = args.q[i];
     // ------------------------------------------------------------- dequant
+    // Group grp handles the iterations it = grp, grp + 4, ... (all in ring
+    // stage s = grp); each thread turns one whole NF4 block (64 weights,
+    // one scale) into bf16 per iteration.
     if (AMODE == A_DEQ_K) {
-      // Row rl of the tile = TMEM lane; this warp covers k = 32*half .. +31 of
-      // each 64-wide stage (one half of the row's NF4 block).
-      const int half = dw >> 2;
+      // Thread: tile row rl (= TMEM lane), k = 0..63 of the stage.
       const int rl = q4 * 32 + lane;
       const int64_t n = row0 + rl;
       const bool valid = n < args.wN;
-      const uint32_t taddr = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col + (uint32_t)(half * 16);
-      const int cofs = rl * 32 + ((half ^ ((rl >> 2) & 1)) << 4);  // 32-byte-swizzled code tile
+      const uint32_t taddr = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col + (uint32_t)(grp * 32);
+      const int sw = (rl >> 2) & 1;  // 32-byte swizzle of the code tile
+      const uint8_t* ctile = smem + grp * L::STAGE + kA + L::B + rl * 32;
       uint32_t c2raw = 0;
       float c1v = 0.0f;
-      if (valid && my_kb > 0) {
-        const int64_t f = n * bpr + kb_lo;
+      if (valid && grp < my_kb) {
+        const int64_t f = n * bpr + kb_lo + grp;
         c2raw = __ldg(args.c2 + f);
         c1v = __ldg(args.c1 + (f >> 8));
       }
-      for (int it = 0; it < my_kb; ++it) {
-        const int s = it % kStages;
+      for (int it = grp; it < my_kb; it += kStages) {
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
-        if (valid && it + 1 < my_kb) {  // the next stage's scale, one stage ahead
-          const int64_t f = n * bpr + kb_lo + it + 1;
+        if (valid && it + kStages < my_kb) {  // this group's next scale, one round ahead
+          const int64_t f = n * bpr + kb_lo + it + kStages;
           c2raw = __ldg(args.c2 + f);
           c1v = __ldg(args.c1 + (f >> 8));
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
-        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane)) break;
+        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
         tc_fence_after();
-        if (!warp_wait(full + s, ph, abort_flag, args.status, lane)) break;
-        const uint4 cw = *reinterpret_cast<const uint4*>(smem + s * L::STAGE + kA + L::B + cofs);
+        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(ctile + (sw << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + ((sw ^ 1) << 4));
         uint32_t o[16];
-        nf4_lookup8(cw.x, tab, o + 0);
-        nf4_lookup8(cw.y, tab, o + 4);
-        nf4_lookup8(cw.z, tab, o + 8);
-        nf4_lookup8(cw.w, tab, o + 12);
-        tmem_st16(taddr + (uint32_t)(s * 32), o);
+        nf4_lookup8(c0.x, tab, o + 0);
+        nf4_lookup8(c0.y, tab, o + 4);
+        nf4_lookup8(c0.z, tab, o + 8);
+        nf4_lookup8(c0.w, tab, o + 12);
+        tmem_st16(taddr, o);
+        nf4_lookup8(c1.x, tab, o + 0);
+        nf4_lookup8(c1.y, tab, o + 4);
+        nf4_lookup8(c1.z, tab, o + 8);
+        nf4_lookup8(c1.w, tab, o + 12);
+        tmem_st16(taddr + 16, o);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(afull + s);
+        if (lane == 0) mbar_arrive(afull + grp);
       }
     } else if (AMODE == A_DEQ_MN) {
       // A = W^T in shared memory, MN-major: rows are k (W columns), the
-      // reduction runs over n (W rows).  Thread (u, half): W row n0 + nl,
-      // 32 consecutive k (k_local = 64*mb + 32*half ..) of one NF4 block.
-      const int e = tid - 64;
-      const int u = e & 127, half = e >> 7;
+      // reduction runs over n (W rows).  Thread u of the group: W row
+      // n0 + nl and the 64 k of NF4 block mb (k_local = 64*mb ..).
+      const int u = q4 * 32 + lane;
       const int nl = u & 63, mb = u >> 6;
       const int64_t kblk = (int64_t)(row0 >> 6) + mb;
       const bool kvalid = kblk < bpr;
       const int r8 = nl & 7;
-      const int cofs = nl * 64 + (((2 * mb + half) ^ ((nl >> 1) & 3)) << 4);  // 64-byte-swizzled code tile
-      const int aofs = mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
+      const int swz = (nl >> 1) & 3;  // 64-byte swizzle of the code tile
+      uint8_t* sa = smem + grp * L::STAGE;
+      const uint8_t* ctile = sa + kA + L::B + nl * 64;
+      uint8_t* atile = sa + mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
       uint32_t c2raw = 0;
       float c1v = 0.0f;
       {
-        const int64_t nn = (int64_t)kb_lo * 64 + nl;
-        if (kvalid && nn < args.wN && my_kb > 0) {
+        const int64_t nn = (int64_t)(kb_lo + grp) * 64 + nl;
+        if (kvalid && nn < args.wN && grp < my_kb) {
           const int64_t f = nn * bpr + kblk;
           c2raw = __ldg(args.c2 + f);
           c1v = __ldg(args.c1 + (f >> 8));
         }
       }
-      for (int it = 0; it < my_kb; ++it) {
-        const int s = it % kStages;
+      for (int it = grp; it < my_kb; it += kStages) {
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const int64_t nn = (int64_t)(kb_lo + it) * 64 + nl;
         const bool valid = kvalid && nn < args.wN;
         const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
-        if (it + 1 < my_kb) {
-          const int64_t nx = nn + 64;
+        if (it + kStages < my_kb) {
+          const int64_t nx = nn + 64 * kStages;
           c2raw = 0;
           c1v = 0.0f;
           if (kvalid && nx < args.wN) {
@@ -291,30 +300,32 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
           }
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
-        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane)) break;
-        if (!warp_wait(full + s, ph, abort_flag, args.status, lane)) break;
-        uint8_t* sa = smem + s * L::STAGE;
-        const uint4 cw = *reinterpret_cast<const uint4*>(sa + kA + L::B + cofs);
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
+        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t o[4];
-          nf4_lookup8(words[j], tab, o);
-          const uint32_t c = (uint32_t)(4 * half + j);
-          *reinterpret_cast<uint4*>(sa + aofs + ((c ^ (uint32_t)r8) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int h = 0; h < 2; ++h) {
+          const uint4 cw = *reinterpret_cast<const uint4*>(ctile + (((2 * mb + h) ^ swz) << 4));
+          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t o[4];
+            nf4_lookup8(words[j], tab, o);
+            const uint32_t c = (uint32_t)(4 * h + j);
+            *reinterpret_cast<uint4*>(atile + ((c ^ (uint32_t)r8) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(afull + s);
+        if (lane == 0) mbar_arrive(afull + grp);
       }
     }
     // ------------------------------------------------------------ epilogue
-    // Two warps per lane quarter: warp group g stores columns [g*BN/2, ...).
+    // Four warps per lane quarter: group grp stores columns [grp*BN/4, ...).
     const bool ok = warp_wait(accum, 0, abort_flag, args.status, lane);
     tc_fence_after();
-    const int g = dw >> 2;
-    const int c_lo = BN >= 32 ? g * (BN / 2) : 0;
-    const int c_hi = BN >= 32 ? c_lo + BN / 2 : (g == 0 ? BN : 0);
+    constexpr int kCols = BN >= 64 ? BN / 4 : 16;
+    const int c_lo = grp * kCols;
+    const int c_hi = c_lo + kCols < BN ? c_lo + kCols : BN;
     const int64_t row = row0 + q4 * 32 + lane;
     for (int c = c_lo; c < c_hi; c += 16) {
       uint32_t v[16];
