@@ -231,8 +231,12 @@ struct Nf4BlockTable {
 
 QDEV Nf4BlockTable nf4_block_table(const float (&q)[16], float chat) {
   uint32_t P[8];
+  const float2 cc = make_float2(chat, chat);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) P[j] = pack_bf16x2(__fmul_rn(q[2 * j], chat), __fmul_rn(q[2 * j + 1], chat));
+  for (int j = 0; j < 8; ++j) {
+    const float2 pr = __fmul2_rn(make_float2(q[2 * j], q[2 * j + 1]), cc);  // two RN32 products
+    P[j] = pack_bf16x2(pr.x, pr.y);
+  }
   Nf4BlockTable t;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {

@@ -15,6 +15,12 @@ namespace qnf4 {
 struct Nf4Tables {
   float q[16];
   float t[15];
+  // Code search used by the quantiser: a degree-5 polynomial f(x) with
+  // f(t[i]) in [i + 0.1, i + 0.9], f(-1) >= 0.1, f(1) <= 14.9 and f increasing
+  // on [-1, 1], so that k = round(f(x) - 1/2) is the code of x or one less and
+  // code = k + (x > t[k]).  poly[0] already includes the -1/2.
+  float poly[6];
+  bool poly_ok;  // the conditions above were verified when the tables were built
 };
 
 // Derived once per process on the host, from the normal quantiles.

@@ -13,6 +13,7 @@
 #include <atomic>
 #include <cmath>
 #include <mutex>
+#include <utility>
 
 #include "internal.h"
 
@@ -41,6 +42,61 @@ float round_down_to_float(double v) {
   return f;
 }
 
+// f(x) evaluated the way the kernel does it: Horner in fp32 with fused
+// multiply-adds (poly[0] holds c0 - 1/2).
+float eval_poly_f32(const float* p, float x) {
+  float f = p[5];
+  for (int k = 4; k >= 0; --k) f = std::fmaf(f, x, p[k]);
+  return f + 0.5f;
+}
+
+// Least-squares fit of f through (t[i], i + 1/2) and the anchors (-1, 0.3),
+// (1, 14.7), then a check of the conditions the quantiser relies on.
+void fit_code_polynomial(Nf4Tables& t) {
+  double xs[17], ys[17];
+  for (int i = 0; i < 15; ++i) {
+    xs[i] = t.t[i];
+    ys[i] = i + 0.5;
+  }
+  xs[15] = -1.0, ys[15] = 0.3;
+  xs[16] = 1.0, ys[16] = 14.7;
+  double A[6][7] = {};
+  for (int n = 0; n < 17; ++n) {
+    double pw[6];
+    pw[0] = 1.0;
+    for (int k = 1; k < 6; ++k) pw[k] = pw[k - 1] * xs[n];
+    for (int r = 0; r < 6; ++r) {
+      for (int c = 0; c < 6; ++c) A[r][c] += pw[r] * pw[c];
+      A[r][6] += pw[r] * ys[n];
+    }
+  }
+  for (int c = 0; c < 6; ++c) {  // Gauss-Jordan with partial pivoting
+    int piv = c;
+    for (int r = c + 1; r < 6; ++r)
+      if (std::fabs(A[r][c]) > std::fabs(A[piv][c])) piv = r;
+    for (int k = 0; k < 7; ++k) std::swap(A[c][k], A[piv][k]);
+    for (int r = 0; r < 6; ++r) {
+      if (r == c) continue;
+      const double m = A[r][c] / A[c][c];
+      for (int k = c; k < 7; ++k) A[r][k] -= m * A[c][k];
+    }
+  }
+  for (int k = 0; k < 6; ++k) t.poly[k] = (float)(A[k][6] / A[k][k]);
+  t.poly[0] = (float)((double)t.poly[0] - 0.5);
+  bool ok = eval_poly_f32(t.poly, -1.0f) >= 0.1f && eval_poly_f32(t.poly, 1.0f) <= 14.9f;
+  for (int i = 0; i < 15; ++i) {
+    const float f = eval_poly_f32(t.poly, t.t[i]);
+    ok = ok && f >= i + 0.1f && f <= i + 0.9f;
+  }
+  float prev = eval_poly_f32(t.poly, -1.0f);
+  for (int n = 1; n <= 1 << 16 && ok; ++n) {  // increasing on a fine grid of [-1, 1]
+    const float f = eval_poly_f32(t.poly, -1.0f + 2.0f * (float)n / (float)(1 << 16));
+    ok = f > prev;
+    prev = f;
+  }
+  t.poly_ok = ok;
+}
+
 Nf4Tables build() {
   const long double delta = 1.0L - 0.5L * (1.0L / 32.0L + 1.0L / 30.0L);
   long double lv[16];
@@ -55,6 +111,7 @@ Nf4Tables build() {
   t.q[7] = 0.0f;
   t.q[15] = 1.0f;
   for (int i = 0; i < 15; ++i) t.t[i] = round_down_to_float(((double)t.q[i] + (double)t.q[i + 1]) * 0.5);
+  fit_code_polynomial(t);
   return t;
 }
 

@@ -14,108 +14,112 @@ constexpr int kGroupBlocks = 256;                 // first-level blocks per c1 s
 constexpr int kQuantThreads = 256;
 
 struct QuantParams {
-  float t[15];  // decision thresholds, RD32 of the level midpoints
+  float t[15];    // decision thresholds, RD32 of the level midpoints
+  float poly[6];  // code-search polynomial (see Nf4Tables)
 };
 
-QDEV uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+constexpr uint32_t kMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23: adding it rounds to an integer
 
-// x = RN32(w / c) for |w| <= c.  For c in [2^-90, 2^100) a correctly rounded
-// reciprocal, one product and one fused correction step give the IEEE
-// quotient's NF4 code for every bf16 pair (checked exhaustively); other
-// finite scales use the IEEE division directly.  A zero or non-finite scale
-// gives x = 0 (a non-finite block is reported through the status word).
-QDEV float ratio(float w, float c, float rc, bool fast) {
-  if (fast) {
-    const float q0 = __fmul_rn(w, rc);
-    const float e = __fmaf_rn(-q0, c, w);
-    return __fmaf_rn(e, rc, q0);
-  }
+// x = RN32(w / c) for a pair of weights against one block scale c.  For c in
+// [2^-90, 2^100) a correctly rounded reciprocal, one product and one fused
+// correction step give the IEEE quotient's NF4 code for every bf16 pair
+// (checked exhaustively on the host); the other scales take the IEEE division.
+// A zero or non-finite scale gives x = 0 (a non-finite block is reported
+// through the status word).
+QDEV float2 ratio_fast(float2 w, float2 c, float2 rc) {
+  const float2 q0 = __fmul2_rn(w, rc);
+  const float2 e = __ffma2_rn(q0, make_float2(-c.x, -c.y), w);
+  return __ffma2_rn(e, rc, q0);
+}
+QDEV float ratio_slow(float w, float c) {
   return (c > 0.0f && c <= 3.402823466e38f) ? __fdiv_rn(w, c) : 0.0f;
 }
 
-// Code of x via a 129-entry bucket table: bucket j = RN(64 x) + 64 covers the
-// closed interval [(j - 64.5)/64, (j - 63.5)/64], which holds at most one
-// threshold (thresholds are >= 0.079 apart).  Entry: (that threshold or +2,
-// number of thresholds below the bucket).
-QDEV uint32_t nf4_code(float x, const float2* bucket) {
-  const float y = __fmaf_rn(x, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64
-  const int j = __float_as_int(y) - 0x4B400000;       // bits of 1.5 * 2^23
-  const float2 b = bucket[min((unsigned)j, 128u)];     // |x| <= 1 keeps j in [0, 128]
-  return (uint32_t)__float_as_int(b.y) + (x > b.x ? 1u : 0u);
+// NF4 codes of a pair x (|x| <= 1): k = round(f(x) - 1/2) is the code or one
+// less (f: the code-search polynomial), and code = k + (x > t[k]).  Returned
+// packed as (code_lo | code_hi << 4).
+QDEV uint32_t nf4_code_pair(float2 x, const float2 (&P)[6], const float* s_t) {
+  float2 f = __ffma2_rn(P[5], x, P[4]);
+  f = __ffma2_rn(f, x, P[3]);
+  f = __ffma2_rn(f, x, P[2]);
+  f = __ffma2_rn(f, x, P[1]);
+  f = __ffma2_rn(f, x, P[0]);
+  const float2 y = __fadd2_rn(f, make_float2(12582912.0f, 12582912.0f));
+  const uint32_t ka = min(__float_as_uint(y.x) - kMagicBits, 14u);  // clamp: no code is ever > 15
+  const uint32_t kb = min(__float_as_uint(y.y) - kMagicBits, 14u);
+  const uint32_t ca = ka + (x.x > s_t[ka] ? 1u : 0u);
+  const uint32_t cb = kb + (x.y > s_t[kb] ? 1u : 0u);
+  return ca | (cb << 4);
 }
 
+// One CTA per 16384-weight group (256 blocks = one c1 scale), 256 threads;
+// 4 threads share a 64-weight block, 16 weights (32 bytes) each, 4 rounds.
 __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint16_t* __restrict__ W,
                                                                       int64_t n_blocks,
-                                                                      uint32_t* __restrict__ codes,
+                                                                      uint2* __restrict__ codes,
                                                                       uint8_t* __restrict__ c2,
                                                                       float* __restrict__ c1, int* status,
                                                                       QuantParams qp) {
-  __shared__ float2 s_bucket[129];
+  __shared__ float s_t[16];
   __shared__ float s_absmax[kGroupBlocks];
   __shared__ float s_wmax[kQuantThreads / 32];
   const int t = threadIdx.x;
-  if (t < 129) {
-    const float lo = ((float)t - 64.5f) * 0.015625f;
-    const float hi = ((float)t - 63.5f) * 0.015625f;
-    int base = 0;
-    float th = 2.0f;
-    for (int i = 0; i < 15; ++i) {
-      if (qp.t[i] < lo) ++base;
-      else if (qp.t[i] <= hi) th = qp.t[i];
-    }
-    s_bucket[t] = make_float2(th, __int_as_float(base));
-  }
+  if (t < 16) s_t[t] = t < 15 ? qp.t[t] : 2.0f;
+  float2 P[6];
+#pragma unroll
+  for (int k = 0; k < 6; ++k) P[k] = make_float2(qp.poly[k], qp.poly[k]);
   __syncthreads();
 
   const int64_t n_groups = (n_blocks + kGroupBlocks - 1) / kGroupBlocks;
   for (int64_t g = blockIdx.x; g < n_groups; g += gridDim.x) {
     const int64_t blk0 = g * kGroupBlocks;
     const int nblk = (int)min((int64_t)kGroupBlocks, n_blocks - blk0);
-    // 8 rounds; in round i thread t owns 8 consecutive weights of block
-    // i*32 + t/8 (16-byte chunk i*256 + t of the group).
+    // round i: unit u = i*256 + t holds 16 weights of block u/4 (part u%4)
     uint4 v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ci = i * kQuantThreads + t;
-      if ((ci >> 3) < nblk) v[i] = ld_stream_v4(W + (blk0 * 64 + (int64_t)ci * 8));
-      else v[i] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 4; ++i) {
+      const int u = i * kQuantThreads + t;
+      if ((u >> 2) < nblk) {
+        const uint4* p = reinterpret_cast<const uint4*>(W + (blk0 * 64 + (int64_t)u * 16));
+        v[2 * i] = __ldg(p);
+        v[2 * i + 1] = __ldg(p + 1);
+      } else {
+        v[2 * i] = v[2 * i + 1] = make_uint4(0, 0, 0, 0);
+      }
     }
     uint32_t bad = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ci = i * kQuantThreads + t;
-      const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    for (int i = 0; i < 4; ++i) {
+      const int u = i * kQuantThreads + t;
+      const uint32_t w8[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
+                              v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
       uint32_t m2 = 0;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t a = w4[k] & 0x7FFF7FFFu;  // |w| as sign-magnitude bits
-        bad |= ((a & 0x7F800000u) == 0x7F800000u) | ((a & 0x7F80u) == 0x7F80u);
-        m2 = __vmaxu2(m2, a);
-      }
+      for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, w8[k] & 0x7FFF7FFFu);  // |w| as sign-magnitude bits
       uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+      bad |= (m >= 0x7F80u) ? 1u : 0u;  // Inf or NaN in the block
       const float c = bf16_bits_to_float(m);
-      if ((t & 7) == 0 && (ci >> 3) < nblk) s_absmax[ci >> 3] = c;
+      if ((t & 3) == 0 && (u >> 2) < nblk) s_absmax[u >> 2] = c;
       const bool fast = c >= 0x1p-90f && c < 0x1p100f;
-      const float rc = fast ? __frcp_rn(c) : 0.0f;
-      uint32_t packed = 0;
+      uint32_t out[2] = {0u, 0u};
+      if (__all_sync(0xFFFFFFFFu, fast)) {
+        const float rc = __frcp_rn(c);
+        const float2 rc2 = make_float2(rc, rc), cc = make_float2(c, c);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float w0 = bf16_bits_to_float(w4[k] & 0xFFFFu);
-        const float w1 = bf16_bits_to_float(w4[k] >> 16);
-        const uint32_t q0 = nf4_code(ratio(w0, c, rc, fast), s_bucket);
-        const uint32_t q1 = nf4_code(ratio(w1, c, rc, fast), s_bucket);
-        packed |= (q0 | (q1 << 4)) << (8 * k);
+        for (int k = 0; k < 8; ++k) {
+          const float2 w = make_float2(__uint_as_float(w8[k] << 16), __uint_as_float(w8[k] & 0xFFFF0000u));
+          out[k >> 2] |= nf4_code_pair(ratio_fast(w, cc, rc2), P, s_t) << (8 * (k & 3));
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float w0 = __uint_as_float(w8[k] << 16), w1 = __uint_as_float(w8[k] & 0xFFFF0000u);
+          out[k >> 2] |= nf4_code_pair(make_float2(ratio_slow(w0, c), ratio_slow(w1, c)), P, s_t) << (8 * (k & 3));
+        }
       }
-      if ((ci >> 3) < nblk) codes[blk0 * 8 + ci] = packed;
+      if ((u >> 2) < nblk) codes[blk0 * 4 + u] = make_uint2(out[0], out[1]);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (t & 31) == 0) report(status, QLORA_ERR_NONFINITE);
     __syncthreads();
@@ -141,39 +145,45 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
 }
 
 // doubleDequant: w^ = RNbf16(RN32(q[code] * RN32(dec(c2) * c1))).
-// Thread handles 8 weights (one 32-bit code word, one 16-byte output) per
-// step, 4 steps per loop trip for memory-level parallelism.
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ codes,
+// A thread turns 32 weights (16 bytes of codes, half an NF4 block) into 64
+// bytes of bf16 per step, two steps per loop trip for memory parallelism.
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4* __restrict__ codes,
                                                           const uint8_t* __restrict__ c2,
-                                                          const float* __restrict__ c1, int64_t n_chunks,
+                                                          const float* __restrict__ c1, int64_t n_units,
                                                           uint4* __restrict__ out, Nf4Tables tab) {
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = tab.q[threadIdx.x];
   __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < n_chunks; c0 += 4 * stride) {
-    uint32_t cw[4];
-    float chat[4];
+  for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < n_units; u0 += 2 * stride) {
+    uint4 cw[2];
+    float chat[2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t ci = c0 + u * stride;
-      if (ci < n_chunks) {
-        cw[u] = __ldcs(codes + ci);
-        const int64_t blk = ci >> 3;
-        chat[u] = decode_scale(__ldg(c2 + blk), __ldg(c1 + (blk >> 8)));
+    for (int h = 0; h < 2; ++h) {
+      const int64_t u = u0 + h * stride;
+      if (u < n_units) {
+        cw[h] = __ldcs(codes + u);
+        const int64_t blk = u >> 1;  // 32 weights per unit, 64 per block
+        chat[h] = decode_scale(__ldg(c2 + blk), __ldg(c1 + (blk >> 8)));
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t ci = c0 + u * stride;
-      if (ci < n_chunks) {
-        uint32_t o[4];
+    for (int h = 0; h < 2; ++h) {
+      const int64_t u = u0 + h * stride;
+      if (u < n_units) {
+        const uint32_t w4[4] = {cw[h].x, cw[h].y, cw[h].z, cw[h].w};
+        const float2 cc = make_float2(chat[h], chat[h]);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint32_t b = cw[u] >> (8 * k);
-          o[k] = pack_bf16x2(__fmul_rn(lut[b & 15u], chat[u]), __fmul_rn(lut[(b >> 4) & 15u], chat[u]));
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t b = w4[k] >> (8 * j);
+            const float2 pr = __fmul2_rn(make_float2(lut[b & 15u], lut[(b >> 4) & 15u]), cc);
+            o[j] = pack_bf16x2(pr.x, pr.y);
+          }
+          __stcs(out + u * 4 + k, make_uint4(o[0], o[1], o[2], o[3]));
         }
-        __stcs(out + ci, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
   }
@@ -200,9 +210,11 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes
   const int64_t n_groups = (n_blocks + kGroupBlocks - 1) / kGroupBlocks;
   QuantParams qp;
   const Nf4Tables& tab = nf4_tables();
+  if (!tab.poly_ok) return cudaErrorNotSupported;
   for (int i = 0; i < 15; ++i) qp.t[i] = tab.t[i];
+  for (int k = 0; k < 6; ++k) qp.poly[k] = tab.poly[k];
   const int64_t grid = n_groups < (int64_t)num_sms() * 16 ? n_groups : (int64_t)num_sms() * 16;
-  nf4_quantize_kernel<<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint32_t*>(codes),
+  nf4_quantize_kernel<<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint2*>(codes),
                                                                  c2, c1, status, qp);
   count_launches(1);
   return cudaGetLastError();
@@ -210,11 +222,11 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
                            uint16_t* out, cudaStream_t st) {
-  const int64_t n_chunks = n_weights / 8;
-  const int64_t want = (n_chunks + 1023) / 1024;
+  const int64_t n_units = n_weights / 32;
+  const int64_t want = (n_units + 511) / 512;
   const int64_t cap = (int64_t)num_sms() * 8;
   const int64_t grid = want < cap ? (want > 0 ? want : 1) : cap;
-  nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes), c2, c1, n_chunks,
+  nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), c2, c1, n_units,
                                                      reinterpret_cast<uint4*>(out), nf4_tables());
   count_launches(1);
   return cudaGetLastError();
