@@ -218,6 +218,43 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def gemv_rates(q, WL, dev, hbm_gbs, pk_kind, copies=4, reps=20):
+    """Forward of the LLaMA-65B FFN up (22016x8192) and down (8192x22016)
+    linears at M = 1, 4, 16 tokens (r = 64), weights rotated over `copies`
+    NF4 copies so that they stream from HBM.  Rate = NF4 weight bytes
+    (codes + c2 + c1) per second of the whole forward call."""
+    import torch
+    wl = WL.WORKLOADS["llama65b_ffn_gemv"]
+    res = {}
+    for lin in wl.linears:
+        t = WL.make_linear(wl, lin, seed=0, device=dev, M=16)
+        ws = [q.quantize(t["W"]) for _ in range(copies)]
+        del t["W"]
+        nbytes = sum(q.storage_bytes(lin.N, lin.K))
+        for M in (1, 4, 16):
+            X = t["X"][:M].contiguous()
+            wsb = torch.empty(q.workspace_bytes(M, lin.N, lin.K, wl.r), dtype=torch.uint8, device=dev)
+            Y = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
+            T = torch.empty((M, wl.r), dtype=torch.float32, device=dev)
+            for i in range(copies):
+                q.linear_fwd(X, ws[i], t["L1"], t["L2"], wl.s, ws=wsb, Y=Y, T=T)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(reps):
+                q.linear_fwd(X, ws[i % copies], t["L1"], t["L2"], wl.s, ws=wsb, Y=Y, T=T)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            gbs = nbytes / (us * 1e-6) / 1e9
+            res[f"{lin.name}_M{M}"] = {"us": us, "weight_gbs": gbs, "frac": gbs / hbm_gbs}
+        del ws
+    res["peak"] = hbm_gbs
+    res["peak_source"] = f"{pk_kind} HBM copy"
+    res["bytes"] = "NF4 codes + c2 + c1 of the linear (0.516 B per weight)"
+    return res
+
+
 # ------------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -346,6 +383,9 @@ def run_ours(args):
     del Wdeq, wq
     assert q.read_status(dev) == 0
 
+    # ---- few-token forward (dequant-GEMV regime): LLaMA-65B FFN up and down
+    gemv = gemv_rates(q, WL, dev, pk["hbm_gbs"], pk_kind) if not args.no_gemv else None
+
     # ---- end to end through the C ABI: activations in, adapter grads out
     pin = lambda t: t.detach().cpu().pin_memory()
     hX = [pin(L["X"]) for L in layers]
@@ -396,6 +436,7 @@ def run_ours(args):
                       "bytes": qb, "peak_source": f"{pk_kind} HBM copy"},
             "dequant": {"value": dequant_gbs, "unit": "GB/s", "frac": dequant_gbs / hbm, "peak": hbm,
                         "bytes": db, "peak_source": f"{pk_kind} HBM copy"},
+            "gemv": gemv,
             "cpu_baseline": base,
             "clocks": clk,
             "gpu_launches": launches,
@@ -445,6 +486,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--profile", action="store_true", help="run the single-linear ncu capture case")
     args = ap.parse_args(argv)
     if args.profile:

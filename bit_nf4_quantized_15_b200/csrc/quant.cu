@@ -35,21 +35,36 @@ QDEV float ratio_slow(float w, float c) {
   return (c > 0.0f && c <= 3.402823466e38f) ? __fdiv_rn(w, c) : 0.0f;
 }
 
-// NF4 codes of a pair x (|x| <= 1): k = round(f(x) - 1/2) is the code or one
-// less (f: the code-search polynomial), and code = k + (x > t[k]).  Returned
-// packed as (code_lo | code_hi << 4).
-QDEV uint32_t nf4_code_pair(float2 x, const float2 (&P)[6], const float* s_t) {
-  float2 f = __ffma2_rn(P[5], x, P[4]);
-  f = __ffma2_rn(f, x, P[3]);
-  f = __ffma2_rn(f, x, P[2]);
-  f = __ffma2_rn(f, x, P[1]);
-  f = __ffma2_rn(f, x, P[0]);
-  const float2 y = __fadd2_rn(f, make_float2(12582912.0f, 12582912.0f));
-  const uint32_t ka = min(__float_as_uint(y.x) - kMagicBits, 14u);  // clamp: no code is ever > 15
-  const uint32_t kb = min(__float_as_uint(y.y) - kMagicBits, 14u);
-  const uint32_t ca = ka + (x.x > s_t[ka] ? 1u : 0u);
-  const uint32_t cb = kb + (x.y > s_t[kb] ? 1u : 0u);
-  return ca | (cb << 4);
+QDEV float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+// NF4 codes of four pairs x[0..3] (|x| <= 1), packed as 8 nibbles (pair j
+// -> nibbles 2j, 2j+1).  k = round(f(x) - 1/2) is the code or one less (f:
+// the code-search polynomial) and code = k + (x > t[k]).  Adding 1.5 * 2^23
+// leaves k in the low bits of the float, so the nibbles are accumulated
+// straight from those bits and the constant part is removed once at the end.
+// The table address is masked to the 16-entry table whatever the input.
+QDEV uint32_t nf4_codes8(const float2 (&x)[4], const float2 (&P)[6], uint32_t t_addr) {
+  uint32_t acc = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float2 f = __ffma2_rn(P[5], x[j], P[4]);
+    f = __ffma2_rn(f, x[j], P[3]);
+    f = __ffma2_rn(f, x[j], P[2]);
+    f = __ffma2_rn(f, x[j], P[1]);
+    f = __ffma2_rn(f, x[j], P[0]);
+    const float2 y = __fadd2_rn(f, make_float2(12582912.0f, 12582912.0f));
+    const uint32_t ba = __float_as_uint(y.x), bb = __float_as_uint(y.y);
+    acc += ba * (1u << (8 * j)) + bb * (1u << (8 * j + 4));
+    const float ta = lds_f32(t_addr + ((ba << 2) & 0x3Cu));
+    const float tb = lds_f32(t_addr + ((bb << 2) & 0x3Cu));
+    if (x[j].x > ta) acc += 1u << (8 * j);
+    if (x[j].y > tb) acc += 1u << (8 * j + 4);
+  }
+  return acc - kMagicBits * 0x11111111u;  // remove sum_i magic * 16^i (mod 2^32)
 }
 
 // One CTA per 16384-weight group (256 blocks = one c1 scale), 256 threads;
@@ -68,6 +83,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
   float2 P[6];
 #pragma unroll
   for (int k = 0; k < 6; ++k) P[k] = make_float2(qp.poly[k], qp.poly[k]);
+  const uint32_t t_addr = smem_u32(s_t);
   __syncthreads();
 
   const int64_t n_groups = (n_blocks + kGroupBlocks - 1) / kGroupBlocks;
@@ -93,32 +109,35 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
       const int u = i * kQuantThreads + t;
       const uint32_t w8[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
-      uint32_t m2 = 0;
+      // |w| max with NaN propagation (bf16x2), then over the 4 threads of the block
+      __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w8[0]));
 #pragma unroll
-      for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, w8[k] & 0x7FFF7FFFu);  // |w| as sign-magnitude bits
-      uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+      for (int k = 1; k < 8; ++k) m2 = __hmax2_nan(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w8[k])));
+      const uint32_t mb = *reinterpret_cast<uint32_t*>(&m2);
+      uint32_t m = max(mb & 0xFFFFu, mb >> 16);  // sign-cleared bits: integer order = magnitude, NaN highest
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
       bad |= (m >= 0x7F80u) ? 1u : 0u;  // Inf or NaN in the block
       const float c = bf16_bits_to_float(m);
       if ((t & 3) == 0 && (u >> 2) < nblk) s_absmax[u >> 2] = c;
       const bool fast = c >= 0x1p-90f && c < 0x1p100f;
-      uint32_t out[2] = {0u, 0u};
+      uint32_t out[2];
+      float2 x[2][4];
       if (__all_sync(0xFFFFFFFFu, fast)) {
         const float rc = __frcp_rn(c);
         const float2 rc2 = make_float2(rc, rc), cc = make_float2(c, c);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float2 w = make_float2(__uint_as_float(w8[k] << 16), __uint_as_float(w8[k] & 0xFFFF0000u));
-          out[k >> 2] |= nf4_code_pair(ratio_fast(w, cc, rc2), P, s_t) << (8 * (k & 3));
-        }
+        for (int k = 0; k < 8; ++k)
+          x[k >> 2][k & 3] = ratio_fast(make_float2(__uint_as_float(w8[k] << 16), __uint_as_float(w8[k] & 0xFFFF0000u)),
+                                        cc, rc2);
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float w0 = __uint_as_float(w8[k] << 16), w1 = __uint_as_float(w8[k] & 0xFFFF0000u);
-          out[k >> 2] |= nf4_code_pair(make_float2(ratio_slow(w0, c), ratio_slow(w1, c)), P, s_t) << (8 * (k & 3));
-        }
+        for (int k = 0; k < 8; ++k)
+          x[k >> 2][k & 3] = make_float2(ratio_slow(__uint_as_float(w8[k] << 16), c),
+                                         ratio_slow(__uint_as_float(w8[k] & 0xFFFF0000u), c));
       }
+      out[0] = nf4_codes8(x[0], P, t_addr);
+      out[1] = nf4_codes8(x[1], P, t_addr);
       if ((u >> 2) < nblk) codes[blk0 * 4 + u] = make_uint2(out[0], out[1]);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (t & 31) == 0) report(status, QLORA_ERR_NONFINITE);
@@ -145,45 +164,47 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
 }
 
 // doubleDequant: w^ = RNbf16(RN32(q[code] * RN32(dec(c2) * c1))).
-// A thread turns 32 weights (16 bytes of codes, half an NF4 block) into 64
-// bytes of bf16 per step, two steps per loop trip for memory parallelism.
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4* __restrict__ codes,
+// A thread turns 8 weights (one 32-bit code word) into one 16-byte bf16
+// store per step; consecutive threads take consecutive words (coalesced), and
+// 8 steps per loop trip keep 8 loads in flight per thread.
+constexpr int kDeqSteps = 8;
+
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ codes,
                                                           const uint8_t* __restrict__ c2,
-                                                          const float* __restrict__ c1, int64_t n_units,
+                                                          const float* __restrict__ c1, int64_t n_chunks,
                                                           uint4* __restrict__ out, Nf4Tables tab) {
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = tab.q[threadIdx.x];
   __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < n_units; u0 += 2 * stride) {
-    uint4 cw[2];
-    float chat[2];
+  for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < n_chunks; c0 += kDeqSteps * stride) {
+    uint32_t cw[kDeqSteps];
+    uint32_t s2[kDeqSteps];
+    float s1[kDeqSteps];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t u = u0 + h * stride;
-      if (u < n_units) {
-        cw[h] = __ldcs(codes + u);
-        const int64_t blk = u >> 1;  // 32 weights per unit, 64 per block
-        chat[h] = decode_scale(__ldg(c2 + blk), __ldg(c1 + (blk >> 8)));
+    for (int u = 0; u < kDeqSteps; ++u) {
+      const int64_t ci = c0 + u * stride;
+      if (ci < n_chunks) {
+        cw[u] = __ldcs(codes + ci);
+        const int64_t blk = ci >> 3;
+        s2[u] = __ldg(c2 + blk);
+        s1[u] = __ldg(c1 + (blk >> 8));
       }
     }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t u = u0 + h * stride;
-      if (u < n_units) {
-        const uint32_t w4[4] = {cw[h].x, cw[h].y, cw[h].z, cw[h].w};
-        const float2 cc = make_float2(chat[h], chat[h]);
+    for (int u = 0; u < kDeqSteps; ++u) {
+      const int64_t ci = c0 + u * stride;
+      if (ci < n_chunks) {
+        const float chat = decode_scale(s2[u], s1[u]);
+        const float2 cc = make_float2(chat, chat);
+        uint32_t o[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t b = w4[k] >> (8 * j);
-            const float2 pr = __fmul2_rn(make_float2(lut[b & 15u], lut[(b >> 4) & 15u]), cc);
-            o[j] = pack_bf16x2(pr.x, pr.y);
-          }
-          __stcs(out + u * 4 + k, make_uint4(o[0], o[1], o[2], o[3]));
+          const uint32_t b = cw[u] >> (8 * k);
+          const float2 pr = __fmul2_rn(make_float2(lut[b & 15u], lut[(b >> 4) & 15u]), cc);
+          o[k] = pack_bf16x2(pr.x, pr.y);
         }
+        __stcs(out + ci, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
   }
@@ -222,11 +243,11 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
                            uint16_t* out, cudaStream_t st) {
-  const int64_t n_units = n_weights / 32;
-  const int64_t want = (n_units + 511) / 512;
+  const int64_t n_chunks = n_weights / 8;
+  const int64_t want = (n_chunks + 256 * kDeqSteps - 1) / (256 * kDeqSteps);
   const int64_t cap = (int64_t)num_sms() * 8;
   const int64_t grid = want < cap ? (want > 0 ? want : 1) : cap;
-  nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), c2, c1, n_units,
+  nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes), c2, c1, n_chunks,
                                                      reinterpret_cast<uint4*>(out), nf4_tables());
   count_launches(1);
   return cudaGetLastError();
