@@ -67,6 +67,8 @@ def oracle_ref(X, W, L1, L2, dY, s, backward=True):
 SHAPES = [  # M, N, K, r: single tiles, ragged tails, split reductions, every token-tile width
     (1, 64, 64, 16), (5, 200, 320, 16), (16, 512, 1024, 64), (37, 136, 256, 32), (64, 128, 128, 48),
     (100, 264, 704, 64), (200, 384, 512, 128), (300, 256, 192, 16), (513, 1000, 640, 64), (1024, 1024, 2048, 64),
+    # several tiles per persistent CTA, each ending with a LoRA extension stage
+    (2048, 4096, 512, 32), (1536, 2560, 1024, 64),
 ]
 
 
