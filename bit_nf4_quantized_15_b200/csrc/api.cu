@@ -108,9 +108,6 @@ void fill_common(EngineArgs* a, int* status) {
 // Launch the engine and, for a split reduction, the fixed-order sum.
 int run(EngineArgs& a, int amode, const GemmPlan& p, float* partial, cudaStream_t st) {
   a.splits = p.splits;
-  a.m_tiles = p.m_tiles;
-  a.n_tiles = p.n_tiles;
-  a.total_tiles = p.m_tiles * p.n_tiles * p.splits;
   a.partial = p.splits > 1 ? partial : nullptr;
   if (launch_engine(a, amode, p, st) != cudaSuccess) return QLORA_ERR_CUDA;
   if (p.splits > 1 && launch_split_reduce(partial, p.splits, a.rows, a.cols, a.epi, st) != cudaSuccess)
@@ -149,12 +146,12 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   w.ofs_sdT = mr;
   w.ofs_partial = 2 * mr;
   const int kbK = (int)(K / 64), kbN = (int)((N + 63) / 64), kbM = (int)((M + 63) / 64);
-  w.t_fwd = plan_gemm((int)M, r, kbK, sms, A_TMA);
-  w.y_fwd = plan_gemm((int)N, (int)M, kbK, sms, A_DEQ_K);
-  w.dt = plan_gemm((int)M, r, kbN, sms, A_TMA);
-  w.dx = plan_gemm((int)K, (int)M, kbN, sms, A_DEQ_MN);
-  w.dl1 = plan_gemm((int)K, r, kbM, sms, A_TMA);
-  w.dl2 = plan_gemm((int)N, r, kbM, sms, A_TMA);
+  w.t_fwd = plan_gemm((int)M, r, kbK, sms);
+  w.y_fwd = plan_gemm((int)N, (int)M, kbK, sms);
+  w.dt = plan_gemm((int)M, r, kbN, sms);
+  w.dx = plan_gemm((int)K, (int)M, kbN, sms);
+  w.dl1 = plan_gemm((int)K, r, kbM, sms);
+  w.dl2 = plan_gemm((int)N, r, kbM, sms);
   size_t part = 0;
   for (const GemmPlan* p : {&w.t_fwd, &w.y_fwd, &w.dt, &w.dx, &w.dl1, &w.dl2})
     part = p->partial_bytes > part ? p->partial_bytes : part;

@@ -60,35 +60,23 @@ QDEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Same, but the thread may be suspended in hardware (up to about a
-// millisecond) until the phase completes instead of returning at once, so a
-// waiting warp does not take issue slots from the warps doing work.
-QDEV bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(1000000u)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase with the given parity to complete.  Bounded: returns
 // false (after flagging the CTA and the caller's status) on timeout or when
-// another role of the CTA has already aborted.
+// another role of the CTA has already aborted.  Plain polling: a suspended
+// wait (try_wait with a time hint) was measured to wake up late.
 QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (;;) {
-    if (mbar_try_wait_suspend(a, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > QNF4_WAIT_NS) {
-      *abort_flag = 1;
-      report(status, QLORA_ERR_TIMEOUT);
-      return false;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > QNF4_WAIT_NS) {
+        *abort_flag = 1;
+        report(status, QLORA_ERR_TIMEOUT);
+        return false;
+      }
     }
   }
 }

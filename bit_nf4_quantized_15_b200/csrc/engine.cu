@@ -2,31 +2,23 @@
 //
 //   D[rows x cols] (fp32, in TMEM) = sum_k A[row, k] * B[col, k]
 //
-// Persistent: one CTA per SM walks a static round-robin list of 128 x BN
-// output tiles (cta_group::1 UMMA, M = 128).  The reduction of every tile
-// runs in 64-wide blocks through one 4-stage shared-memory ring that keeps
-// flowing from tile to tile:
+// One CTA computes a 128 x BN output tile with cta_group::1 UMMA (M = 128).
+// The reduction runs in 64-wide blocks through a 4-stage shared-memory ring:
 //   * warp 0, one lane: TMA producer (B tiles, A tiles or NF4 code tiles);
 //   * warp 1, one lane: UMMA issuer, 4 x (128 x BN x 16) MMAs per stage,
-//     tcgen05.commit frees the stage and, after a tile's last stage, hands
-//     the accumulator to the epilogue;
-//   * warps 2..17, four groups of four: when A is the NF4 weight, group g
-//     turns the code tile of ring stage g into bf16 (one NF4 block per thread)
-//     -- into tensor memory for X.W^T, into the 128-byte-swizzled MN-major
-//     shared-memory layout for dY.W;
-//   * warps 18..21: epilogue (TMEM -> registers -> global).  With two
-//     accumulators in TMEM the epilogue of one tile overlaps the MMAs of the
-//     next.
+//     tcgen05.commit frees the stage;
+//   * warps 2..5 (128 threads): when A is the NF4 weight, they turn the code
+//     tile into a bf16 tile in the 128-byte-swizzled canonical layout UMMA
+//     reads (K-major for X.W^T, MN-major for dY.W), then run the epilogue
+//     (TMEM -> registers -> global, one accumulator row per thread).
 // An optional extension segment appends more reduction blocks from other
 // operands into the same accumulator: this is how the LoRA term s.T.L2
 // (forward) and s.dT.L1^T (backward) is added to the dequantised product.
-// A split of the main reduction writes fp32 partial tiles that a second
-// kernel sums in a fixed order (deterministic).
+// A split of the main reduction over grid.z writes fp32 partial tiles that
+// a second kernel sums in a fixed order (deterministic).
 //
 // inferensys glossary "QLoRA", kernel paragraph: 4-bit weights are loaded,
-// decompressed on chip and fed to the tensor cores as BFloat16.
-#include <cstdlib>
-
+// decompressed in shared memory and fed to the tensor cores as BFloat16.
 #include "common.cuh"
 #include "internal.h"
 
@@ -34,25 +26,20 @@ namespace qnf4 {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kDeqWarps = 16;  // warps 2..17: four groups, group g fills ring stage g
-constexpr int kGroupWarps = 4;
-constexpr int kEpiWarps = 4;   // warps 18..21
-constexpr int kEpiWarp0 = 2 + kDeqWarps;
-constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr int kA = 16384;  // 128 rows x 64 bf16
+constexpr int kDeqWarps = 16;                  // warps 2..17: dequant, then epilogue
+constexpr int kGroupWarps = 4;                 // one group of 4 warps per ring stage
+constexpr int kThreads = 64 + 32 * kDeqWarps;  // + producer warp + UMMA warp
+constexpr int kA = 16384;                      // 128 rows x 64 bf16
 
-constexpr uint32_t pow2_cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
-
-// Tensor-memory columns: n_acc fp32 accumulators of max(BN, 32) columns and,
-// for the forward fused GEMM, the dequantised A tile of every ring stage
+// Tensor-memory columns: the fp32 accumulator (BN columns, at least 32) and,
+// for the forward fused GEMM, the dequantised A tile of every stage
 // (128 lanes x 32 columns: 64 bf16 per lane).
 template <int BN, int AMODE>
 struct Tmem {
   static constexpr uint32_t acc = BN < 32 ? 32 : BN;
-  static constexpr uint32_t a_cols = AMODE == A_DEQ_K ? kStages * 32 : 0;
-  static constexpr int n_acc = (2 * acc + a_cols <= 512) ? 2 : 1;
-  static constexpr uint32_t a_col = n_acc * acc;
-  static constexpr uint32_t cols = pow2_cols(a_col + a_cols);
+  static constexpr uint32_t a_col = acc;
+  static constexpr uint32_t need = acc + (AMODE == A_DEQ_K ? kStages * 32 : 0);
+  static constexpr uint32_t cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 };
 
 template <int BN, int AMODE>
@@ -105,42 +92,6 @@ QDEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, in
   return ok != 0;
 }
 
-// The tile list all roles walk in the same order: tile t = blockIdx.x + i *
-// gridDim.x; the weight-row tile varies fastest, then the token tile, then
-// the split of the reduction.  `it` indexes the reduction blocks of a tile
-// (main blocks first, then the extension blocks of split 0).
-struct TileIter {
-  int t, it;
-  int row0, col0, z, kb_lo, my_kb, n_iters;
-  bool valid;
-
-  QDEV void load(const EngineArgs& a, int BN) {
-    const int mt = t % a.m_tiles;
-    const int r = t / a.m_tiles;
-    const int nt = r % a.n_tiles;
-    z = r / a.n_tiles;
-    row0 = mt * 128;
-    col0 = nt * BN;
-    kb_lo = (int)((int64_t)z * a.kb_main / a.splits);
-    my_kb = (int)((int64_t)(z + 1) * a.kb_main / a.splits) - kb_lo;
-    n_iters = my_kb + (z == 0 ? a.kb_ext : 0);
-  }
-  QDEV void begin(const EngineArgs& a, int BN) {
-    t = blockIdx.x;
-    it = 0;
-    valid = t < a.total_tiles;
-    if (valid) load(a, BN);
-  }
-  QDEV void next(const EngineArgs& a, int BN) {
-    if (++it >= n_iters) {
-      t += gridDim.x;
-      it = 0;
-      valid = t < a.total_tiles;
-      if (valid) load(a, BN);
-    }
-  }
-};
-
 template <int BN, int AMODE>
 __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_constant__ EngineArgs args) {
   using L = Layout<BN, AMODE>;
@@ -150,12 +101,16 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR);
   uint64_t* afull = full + kStages;
   uint64_t* empty = afull + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* accum = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row0 = blockIdx.x * 128, col0 = blockIdx.y * BN, z = blockIdx.z;
+  const int kb_lo = (int)((int64_t)z * args.kb_main / args.splits);
+  const int kb_hi = (int)((int64_t)(z + 1) * args.kb_main / args.splits);
+  const int my_kb = kb_hi - kb_lo;
+  const int n_iters = my_kb + (z == 0 ? args.kb_ext : 0);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -163,10 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
       mbar_init(afull + s, kGroupWarps);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, kEpiWarps);
-    }
+    mbar_init(accum, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -186,33 +138,32 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  bool committed_accum = false;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      TileIter ti;
-      uint32_t G = 0;
-      for (ti.begin(args, BN); ti.valid; ti.next(args, BN), ++G) {
-        const int s = (int)(G % kStages);
-        const uint32_t ph = (G / kStages) & 1u;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
         uint8_t* sa = smem + s * L::STAGE;
         uint8_t* sb = sa + kA;
         uint8_t* sc = sb + L::B;
-        if (ti.it < ti.my_kb) {
-          const int kb = ti.kb_lo + ti.it;
+        if (it < my_kb) {
+          const int kb = kb_lo + it;
           uint32_t bytes = tx_bytes(args.b_mn_main, BN);
           bytes += AMODE == A_TMA ? tx_bytes(args.a_mn_main, 128) : 4096u;
           mbar_arrive_expect_tx(full + s, bytes);
-          if (AMODE == A_DEQ_K) tma_load_2d(sc, &args.tmA, full + s, kb * 32, ti.row0);
-          else if (AMODE == A_DEQ_MN) tma_load_2d(sc, &args.tmA, full + s, ti.row0 / 2, kb * 64);
-          else load_operand(sa, &args.tmA, full + s, args.a_mn_main, ti.row0, kb * 64, 128);
-          load_operand(sb, &args.tmB, full + s, args.b_mn_main, ti.col0, kb * 64, BN);
+          if (AMODE == A_DEQ_K) tma_load_2d(sc, &args.tmA, full + s, kb * 32, row0);
+          else if (AMODE == A_DEQ_MN) tma_load_2d(sc, &args.tmA, full + s, row0 / 2, kb * 64);
+          else load_operand(sa, &args.tmA, full + s, args.a_mn_main, row0, kb * 64, 128);
+          load_operand(sb, &args.tmB, full + s, args.b_mn_main, col0, kb * 64, BN);
         } else {
-          const int kb = ti.it - ti.my_kb;
+          const int kb = it - my_kb;
           mbar_arrive_expect_tx(full + s, tx_bytes(args.a_mn_ext, 128) + tx_bytes(args.b_mn_ext, BN));
-          load_operand(sa, &args.tmAx, full + s, args.a_mn_ext, ti.row0, kb * 64, 128);
-          load_operand(sb, &args.tmBx, full + s, args.b_mn_ext, ti.col0, kb * 64, BN);
+          load_operand(sa, &args.tmAx, full + s, args.a_mn_ext, row0, kb * 64, 128);
+          load_operand(sb, &args.tmBx, full + s, args.b_mn_ext, col0, kb * 64, BN);
         }
       }
     }
@@ -222,25 +173,12 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
       const int a_mn_main = AMODE == A_DEQ_MN ? 1 : (AMODE == A_DEQ_K ? 0 : args.a_mn_main);
       const uint32_t id_main = idesc_bf16(128, BN, a_mn_main, args.b_mn_main);
       const uint32_t id_ext = idesc_bf16(128, BN, args.a_mn_ext, args.b_mn_ext);
-      TileIter ti;
-      uint32_t G = 0, tile_no = 0, acc_addr = tmem_d;
-      uint32_t aphase = 0;  // afull completes only for main-segment stages: own parity bit per stage
-      bool ok = true;
-      for (ti.begin(args, BN); ti.valid && ok; ti.next(args, BN), ++G) {
-        if (ti.it == 0) {  // new tile: wait until the epilogue has drained this accumulator
-          const uint32_t b = tile_no % TM::n_acc, use = tile_no / TM::n_acc;
-          if (!mbar_wait(acc_empty + b, (use & 1u) ^ 1u, abort_flag, args.status)) break;
-          tc_fence_after();
-          acc_addr = tmem_d + b * TM::acc;
-        }
-        const int s = (int)(G % kStages);
-        const uint32_t ph = (G / kStages) & 1u;
-        const bool ext = ti.it >= ti.my_kb;
-        ok = mbar_wait(full + s, ph, abort_flag, args.status);
-        if (ok && AMODE != A_TMA && !ext) {
-          ok = mbar_wait(afull + s, (aphase >> s) & 1u, abort_flag, args.status);
-          aphase ^= 1u << s;
-        }
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const bool ext = it >= my_kb;
+        bool ok = mbar_wait(full + s, ph, abort_flag, args.status);
+        if (ok && AMODE != A_TMA && !ext) ok = mbar_wait(afull + s, ph, abort_flag, args.status);
         if (!ok) break;
         tc_fence_after();
         const uint8_t* sa = smem + s * L::STAGE;
@@ -250,165 +188,186 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
           const uint32_t a_tmem = tmem_d + TM::a_col + (uint32_t)(s * 32);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_tmem_a(acc_addr, a_tmem + kk * 8, operand_desc(sb, args.b_mn_main, kk), id_main,
-                             (ti.it | kk) != 0);
+            umma_bf16_tmem_a(tmem_d, a_tmem + kk * 8, operand_desc(sb, args.b_mn_main, kk), id_main,
+                             (it | kk) != 0);
         } else {
           const int amn = ext ? args.a_mn_ext : a_mn_main;
           const int bmn = ext ? args.b_mn_ext : args.b_mn_main;
           const uint32_t id = ext ? id_ext : id_main;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(acc_addr, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (ti.it | kk) != 0);
+            umma_bf16(tmem_d, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (it | kk) != 0);
         }
         umma_commit(empty + s);
-        if (ti.it == ti.n_iters - 1) {  // tile complete: hand the accumulator over
-          umma_commit(acc_full + (tile_no % TM::n_acc));
-          ++tile_no;
-        }
       }
+      umma_commit(accum);
+      committed_accum = true;
     }
     __syncwarp();
-  } else if (warp < kEpiWarp0) {
+  } else {
+    const int dw = warp - 2;           // dequant warp 0..15
+    const int q4 = warp & 3;           // TMEM lane quarter this warp may access
+    const int grp = dw >> 2;           // group = the ring stage these 4 warps fill
+    const int64_t bpr = args.wK / 64;  // NF4 blocks per weight row
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = args.q[i];
     // ------------------------------------------------------------- dequant
-    if (AMODE != A_TMA) {
-      const int grp = (warp - 2) >> 2;  // this group fills ring stage grp
-      const int q4 = warp & 3;          // TMEM lane quarter this warp may access
-      const int u = q4 * 32 + lane;     // thread index within the group
-      const int64_t bpr = args.wK / 64; // NF4 blocks per weight row
-      float q[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) q[i] = args.q[i];
-      // Walk the global stage sequence G = grp, grp + 4, ...; dequantise the
-      // main-segment blocks among them.
-      TileIter ti;
-      ti.begin(args, BN);
-      uint32_t G = 0;
-      for (; G < (uint32_t)grp && ti.valid; ++G) ti.next(args, BN);
-      for (; ti.valid;) {
-        const uint32_t ph = (G / kStages) & 1u;
-        if (ti.it >= ti.my_kb) {
-          // Extension stage: A arrives by TMA.  Still pass through this stage's
-          // phases so that no later wait of the group is two phases ahead of a
-          // barrier (a parity wait cannot tell those apart).
-          if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
-          if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
-        } else {
-          const int kb = ti.kb_lo + ti.it;
-          if (AMODE == A_DEQ_K) {
-            // thread u = tile row (= TMEM lane), k = 0..63 of the stage
-            const int64_t n = ti.row0 + u;
-            float chat = 0.0f;
-            if (n < args.wN) {
-              const int64_t f = n * bpr + kb;
-              chat = decode_scale(__ldg(args.c2 + f), __ldg(args.c1 + (f >> 8)));
-            }
-            const Nf4BlockTable tab = nf4_block_table(q, chat);
-            if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
-            tc_fence_after();
-            if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
-            const uint8_t* ctile = smem + grp * L::STAGE + kA + L::B + u * 32;
-            const int sw = (u >> 2) & 1;  // 32-byte swizzle of the code tile
-            const uint4 c0 = *reinterpret_cast<const uint4*>(ctile + (sw << 4));
-            const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + ((sw ^ 1) << 4));
-            const uint32_t taddr = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col + (uint32_t)(grp * 32);
-            uint32_t o[16];
-            nf4_lookup8(c0.x, tab, o + 0);
-            nf4_lookup8(c0.y, tab, o + 4);
-            nf4_lookup8(c0.z, tab, o + 8);
-            nf4_lookup8(c0.w, tab, o + 12);
-            tmem_st16(taddr, o);
-            nf4_lookup8(c1.x, tab, o + 0);
-            nf4_lookup8(c1.y, tab, o + 4);
-            nf4_lookup8(c1.z, tab, o + 8);
-            nf4_lookup8(c1.w, tab, o + 12);
-            tmem_st16(taddr + 16, o);
-            tmem_wait_st();
-            tc_fence_before();
-          } else {
-            // A = W^T in shared memory, MN-major: thread u = (W row n0 + nl,
-            // NF4 block mb of the 128 tile rows), 64 weights.
-            const int nl = u & 63, mb = u >> 6;
-            const int64_t kblk = (int64_t)(ti.row0 >> 6) + mb;
-            const int64_t nn = (int64_t)kb * 64 + nl;
-            float chat = 0.0f;
-            if (kblk < bpr && nn < args.wN) {
-              const int64_t f = nn * bpr + kblk;
-              chat = decode_scale(__ldg(args.c2 + f), __ldg(args.c1 + (f >> 8)));
-            }
-            const Nf4BlockTable tab = nf4_block_table(q, chat);
-            if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
-            if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
-            uint8_t* sa = smem + grp * L::STAGE;
-            const uint8_t* ctile = sa + kA + L::B + nl * 64;
-            const int swz = (nl >> 1) & 3;  // 64-byte swizzle of the code tile
-            const int r8 = nl & 7;
-            uint8_t* atile = sa + mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint4 cw = *reinterpret_cast<const uint4*>(ctile + (((2 * mb + h) ^ swz) << 4));
-              const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                uint32_t o[4];
-                nf4_lookup8(words[j], tab, o);
-                const uint32_t c = (uint32_t)(4 * h + j);
-                *reinterpret_cast<uint4*>(atile + ((c ^ (uint32_t)r8) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-              }
-            }
-            fence_proxy_async_smem();
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(afull + grp);
+    // Group grp handles the iterations it = grp, grp + 4, ... (all in ring
+    // stage s = grp); each thread turns one whole NF4 block (64 weights,
+    // one scale) into bf16 per iteration.
+    if (AMODE == A_DEQ_K) {
+      // Thread: tile row rl (= TMEM lane), k = 0..63 of the stage.
+      const int rl = q4 * 32 + lane;
+      const int64_t n = row0 + rl;
+      const bool valid = n < args.wN;
+      const uint32_t taddr = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col + (uint32_t)(grp * 32);
+      const int sw = (rl >> 2) & 1;  // 32-byte swizzle of the code tile
+      const uint8_t* ctile = smem + grp * L::STAGE + kA + L::B + rl * 32;
+      uint32_t c2raw = 0;
+      float c1v = 0.0f;
+      if (valid && grp < my_kb) {
+        const int64_t f = n * bpr + kb_lo + grp;
+        c2raw = __ldg(args.c2 + f);
+        c1v = __ldg(args.c1 + (f >> 8));
+      }
+      for (int it = grp; it < my_kb; it += kStages) {
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        if (valid && it + kStages < my_kb) {  // this group's next scale, one round ahead
+          const int64_t f = n * bpr + kb_lo + it + kStages;
+          c2raw = __ldg(args.c2 + f);
+          c1v = __ldg(args.c1 + (f >> 8));
         }
-        for (int k = 0; k < kStages && ti.valid; ++k, ++G) ti.next(args, BN);
+        const Nf4BlockTable tab = nf4_block_table(q, chat);
+        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
+        tc_fence_after();
+        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(ctile + (sw << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + ((sw ^ 1) << 4));
+        uint32_t o[16];
+        nf4_lookup8(c0.x, tab, o + 0);
+        nf4_lookup8(c0.y, tab, o + 4);
+        nf4_lookup8(c0.z, tab, o + 8);
+        nf4_lookup8(c0.w, tab, o + 12);
+        tmem_st16(taddr, o);
+        nf4_lookup8(c1.x, tab, o + 0);
+        nf4_lookup8(c1.y, tab, o + 4);
+        nf4_lookup8(c1.z, tab, o + 8);
+        nf4_lookup8(c1.w, tab, o + 12);
+        tmem_st16(taddr + 16, o);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull + grp);
+      }
+    } else if (AMODE == A_DEQ_MN) {
+      // A = W^T in shared memory, MN-major: rows are k (W columns), the
+      // reduction runs over n (W rows).  Thread u of the group: W row
+      // n0 + nl and the 64 k of NF4 block mb (k_local = 64*mb ..).
+      const int u = q4 * 32 + lane;
+      const int nl = u & 63, mb = u >> 6;
+      const int64_t kblk = (int64_t)(row0 >> 6) + mb;
+      const bool kvalid = kblk < bpr;
+      const int r8 = nl & 7;
+      const int swz = (nl >> 1) & 3;  // 64-byte swizzle of the code tile
+      uint8_t* sa = smem + grp * L::STAGE;
+      const uint8_t* ctile = sa + kA + L::B + nl * 64;
+      uint8_t* atile = sa + mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
+      uint32_t c2raw = 0;
+      float c1v = 0.0f;
+      {
+        const int64_t nn = (int64_t)(kb_lo + grp) * 64 + nl;
+        if (kvalid && nn < args.wN && grp < my_kb) {
+          const int64_t f = nn * bpr + kblk;
+          c2raw = __ldg(args.c2 + f);
+          c1v = __ldg(args.c1 + (f >> 8));
+        }
+      }
+      for (int it = grp; it < my_kb; it += kStages) {
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const int64_t nn = (int64_t)(kb_lo + it) * 64 + nl;
+        const bool valid = kvalid && nn < args.wN;
+        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        if (it + kStages < my_kb) {
+          const int64_t nx = nn + 64 * kStages;
+          c2raw = 0;
+          c1v = 0.0f;
+          if (kvalid && nx < args.wN) {
+            const int64_t f = nx * bpr + kblk;
+            c2raw = __ldg(args.c2 + f);
+            c1v = __ldg(args.c1 + (f >> 8));
+          }
+        }
+        const Nf4BlockTable tab = nf4_block_table(q, chat);
+        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
+        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 cw = *reinterpret_cast<const uint4*>(ctile + (((2 * mb + h) ^ swz) << 4));
+          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t o[4];
+            nf4_lookup8(words[j], tab, o);
+            const uint32_t c = (uint32_t)(4 * h + j);
+            *reinterpret_cast<uint4*>(atile + ((c ^ (uint32_t)r8) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull + grp);
       }
     }
-  } else {
     // ------------------------------------------------------------ epilogue
-    const int q4 = warp & 3;
-    uint32_t tile_no = 0;
-    for (int t = blockIdx.x; t < args.total_tiles; t += gridDim.x, ++tile_no) {
-      TileIter ti;
-      ti.t = t;
-      ti.load(args, BN);
-      const uint32_t b = tile_no % TM::n_acc, use = tile_no / TM::n_acc;
-      const bool ok = warp_wait(acc_full + b, use & 1u, abort_flag, args.status, lane);
-      if (!ok) break;
-      tc_fence_after();
-      const int64_t row = ti.row0 + q4 * 32 + lane;
-      const bool row_ok = row < args.rows;
-      const uint32_t tbase = tmem_d + b * TM::acc + ((uint32_t)(q4 * 32) << 16);
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tbase + (uint32_t)c, v);
-        tmem_wait_ld();
-        if (!row_ok) continue;
-        const int ncol = min(16, args.cols - (ti.col0 + c));
-        if (args.splits > 1) {
-          float* dst = args.partial + ((int64_t)ti.z * args.cols + ti.col0 + c) * args.rows + row;
+    // Four warps per lane quarter: group grp stores columns [grp*BN/4, ...).
+    const bool ok = warp_wait(accum, 0, abort_flag, args.status, lane);
+    tc_fence_after();
+    constexpr int kCols = BN >= 64 ? BN / 4 : 16;
+    const int c_lo = grp * kCols;
+    const int c_hi = c_lo + kCols < BN ? c_lo + kCols : BN;
+    const int64_t row = row0 + q4 * 32 + lane;
+    const EpiArgs& e = args.epi;
+    for (int c = c_lo; c < c_hi; c += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem_d + ((uint32_t)(q4 * 32) << 16) + (uint32_t)c, v);
+      tmem_wait_ld();
+      if (!ok || *abort_flag || row >= args.rows) continue;
+      const int64_t col = col0 + c;
+      const int ncol = min(16, args.cols - (int)col);
+      if (args.splits > 1) {
+        float* dst = args.partial + ((int64_t)z * args.cols + col) * args.rows + row;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < ncol) dst[(int64_t)j * args.rows] = __uint_as_float(v[j]);
+      } else {
+        if (e.out) {
+          if (e.out_bf16) {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(e.out) + row * e.rs + col * e.cs;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < ncol) dst[j * e.cs] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(v[j]), e.alpha));
+          } else {
+            float* dst = reinterpret_cast<float*>(e.out) + row * e.rs + col * e.cs;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < ncol) dst[j * e.cs] = __fmul_rn(__uint_as_float(v[j]), e.alpha);
+          }
+        }
+        if (e.out2) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(e.out2) + row * e.rs2 + col * e.cs2;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < ncol) dst[(int64_t)j * args.rows] = __uint_as_float(v[j]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < ncol) epi_store(args.epi, row, ti.col0 + c + j, __uint_as_float(v[j]));
+            if (j < ncol) dst[j * e.cs2] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(v[j]), e.alpha2));
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + b);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (*abort_flag && lane == 0) {  // let in-flight copies and MMAs land before freeing TMEM
-      const uint64_t t0 = globaltimer();
-      while (globaltimer() - t0 < 2000000ull) {
-      }
-    }
+    if (*abort_flag && lane == 0 && committed_accum) mbar_wait_drain(accum, 0, 10000000ull);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_d, TM::cols);
@@ -431,7 +390,7 @@ cudaError_t launch_t(const EngineArgs& a, const GemmPlan& p, cudaStream_t st) {
   auto kern = umma_engine_kernel<BN, AMODE>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
   if (err != cudaSuccess) return err;
-  const int grid = a.total_tiles < p.num_sms ? a.total_tiles : p.num_sms;
+  dim3 grid(p.m_tiles, p.n_tiles, p.splits);
   kern<<<grid, kThreads, L::TOTAL, st>>>(a);
   count_launches(1);
   return cudaGetLastError();
@@ -444,7 +403,6 @@ cudaError_t launch_mode(const EngineArgs& a, const GemmPlan& p, cudaStream_t st)
     case 32: return launch_t<32, AMODE>(a, p, st);
     case 64: return launch_t<64, AMODE>(a, p, st);
     case 128: return launch_t<128, AMODE>(a, p, st);
-    case 192: return launch_t<192, AMODE>(a, p, st);
     case 256: return launch_t<256, AMODE>(a, p, st);
   }
   return cudaErrorInvalidValue;
@@ -452,27 +410,11 @@ cudaError_t launch_mode(const EngineArgs& a, const GemmPlan& p, cudaStream_t st)
 
 }  // namespace
 
-// Widest token tile: 256, or 192 where a second accumulator then fits in
-// tensor memory next to the forward's dequantised A stages
-// (QLORA_NF4_WIDE_BN=256|192 overrides the default for that case).
-int wide_bn(int amode) {
-  if (amode != A_DEQ_K) return 256;
-  static int v = [] {
-    const char* e = std::getenv("QLORA_NF4_WIDE_BN");
-    const int x = e ? std::atoi(e) : 0;
-    return (x == 192 || x == 256) ? x : 256;
-  }();
-  return v;
-}
+int bn_for_cols(int cols) { return cols <= 16 ? 16 : cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : 256; }
 
-int bn_for_cols(int cols, int amode) {
-  return cols <= 16 ? 16 : cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : wide_bn(amode);
-}
-
-GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms, int amode) {
+GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms) {
   GemmPlan p{};
-  p.num_sms = num_sms;
-  p.BN = bn_for_cols(cols, amode);
+  p.BN = bn_for_cols(cols);
   p.m_tiles = (rows + 127) / 128;
   p.n_tiles = (cols + p.BN - 1) / p.BN;
   const int tiles = p.m_tiles * p.n_tiles;

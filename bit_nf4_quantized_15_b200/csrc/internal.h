@@ -60,7 +60,6 @@ struct EngineArgs {
   const float* c1;
   int64_t wN, wK;    // quantised weight shape (for scale indexing)
   int rows, cols;    // output extent: UMMA-M side, UMMA-N side
-  int m_tiles, n_tiles, total_tiles;  // 128-row tiles, BN-column tiles, x splits
   int kb_main;       // 64-wide reduction blocks of the main segment
   int kb_ext;        // 64-wide reduction blocks of the extension (0: none)
   int splits;        // split of the main reduction across grid.z
@@ -74,11 +73,10 @@ struct EngineArgs {
 struct GemmPlan {
   int BN;
   int m_tiles, n_tiles, splits;
-  int num_sms;
   size_t partial_bytes;
 };
 
-GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms, int amode);
+GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms);
 size_t engine_smem_bytes(int BN, int amode);
 cudaError_t launch_engine(const EngineArgs& a, int amode, const GemmPlan& p, cudaStream_t st);
 cudaError_t launch_split_reduce(const float* partial, int splits, int rows, int cols, const EpiArgs& e,
