@@ -452,7 +452,8 @@ def run_profile_case(args):
     """One linear (gate, 11008x4096, 4096 tokens, r = 64): quantise, then two
     forward + backward passes; the second is the one to capture with ncu
     (engine launches in order: T, Y, dT, dX, dL1, dL2).  Then two quantise and
-    two dequantise passes of a 32768x4096 weight."""
+    two dequantise passes of a 32768x4096 weight, then few-token forwards
+    (M = 16, 1, 16, 1) of the LLaMA-65B FFN up linear 22016x8192."""
     import torch
     import bit_nf4_quantized_15_b200 as q
     from bit_nf4_quantized_15_b200 import workloads as WL
@@ -472,6 +473,16 @@ def run_profile_case(args):
         q.quantize_into(Wbig, wbig)
     for _ in range(2):
         q.dequant(wbig, out=out)
+    # then few-token forwards of the 65B FFN up linear (22016x8192): M = 16, 1, 16, 1
+    del Wbig, wbig, out
+    gw = WL.WORKLOADS["llama65b_ffn_gemv"]
+    g = WL.make_linear(gw, gw.linears[0], seed=0, device="cuda", M=16)
+    gq = q.quantize(g["W"])
+    gws = torch.empty(q.workspace_bytes(16, gw.linears[0].N, gw.linears[0].K, gw.r), dtype=torch.uint8,
+                      device="cuda")
+    for _ in range(2):
+        for M in (16, 1):
+            q.linear_fwd(g["X"][:M].contiguous(), gq, g["L1"], g["L2"], gw.s, ws=gws)
     torch.cuda.synchronize()
     assert q.read_status() == 0
     print(json.dumps({"profile_case": f"{lin.name} {lin.N}x{lin.K}", "tokens": wl.M, "r": wl.r,

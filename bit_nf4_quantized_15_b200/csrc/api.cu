@@ -138,6 +138,7 @@ bool valid_rank(int r) { return r >= 16 && r <= 128 && r % 16 == 0; }
 struct WsLayout {
   size_t ofs_sdT, ofs_partial, total;
   GemmPlan t_fwd, y_fwd, dt, dx, dl1, dl2;
+  GemvPlan gemv;  // M <= kGemvMaxM only
 };
 
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
@@ -155,6 +156,11 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t part = 0;
   for (const GemmPlan* p : {&w.t_fwd, &w.y_fwd, &w.dt, &w.dx, &w.dl1, &w.dl2})
     part = p->partial_bytes > part ? p->partial_bytes : part;
+  if (M <= kGemvMaxM) {  // few-token forward: stream-K partials + T slices
+    w.gemv = plan_gemv(M, N, K, sms);
+    const size_t g = align256(w.gemv.part_bytes) + align256(w.gemv.tp_bytes) + w.gemv.stw_bytes;
+    part = g > part ? g : part;
+  }
   w.total = w.ofs_partial + align256(part);
   return w;
 }
@@ -259,6 +265,43 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* sT = reinterpret_cast<uint16_t*>(wsb);
   float* partial = reinterpret_cast<float*>(wsb + lay.ofs_partial);
+
+  if (M <= kGemvMaxM) {
+    // Few tokens: weight-streaming dequant-GEMV (stream-K over all SMs).
+    const GemvPlan& gp = lay.gemv;
+    GemvArgs ga;
+    std::memset(&ga, 0, sizeof(ga));
+    if (make_map(&ga.tmCodes, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+        map_operand(&ga.tmX, X, 0, M, K, 16))
+      return QLORA_ERR_CUDA;
+    ga.c2 = w->c2;
+    ga.c1 = w->c1;
+    ga.N = N;
+    ga.K = K;
+    ga.M = (int)M;
+    ga.kbt = gp.kbt;
+    ga.upr = gp.upr;
+    ga.m_tiles = gp.m_tiles;
+    ga.maxc = gp.maxc;
+    ga.units = gp.units;
+    ga.part = partial;
+    uint8_t* gws = wsb + lay.ofs_partial + align256(gp.part_bytes);
+    ga.tp = reinterpret_cast<float*>(gws);
+    ga.sTw = reinterpret_cast<float*>(gws + align256(gp.tp_bytes));
+    ga.r = r;
+    ga.s = s;
+    ga.T_save = T_save;
+    ga.status = status_dev;
+    const Nf4Tables& tb = nf4_tables();
+    for (int i = 0; i < 16; ++i) ga.q[i] = tb.q[i];
+    cudaEvent_t e0 = g_ev_start, e1 = g_ev_end;
+    g_ev_start = g_ev_end = nullptr;
+    if (e0 && cudaEventRecord(e0, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_gemv(ga, gp, X, L1, L2, Y, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (e1 && cudaEventRecord(e1, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
 
   // (1) T = X.L1 (fp32, saved) and s.T in bf16 for the LoRA extension.
   {

@@ -1,0 +1,603 @@
+// Few-token forward (M <= 16): the dequant-GEMV regime, where the time is the
+// stream of 4-bit weights from HBM (0.516 byte per weight) and the tensor
+// cores have almost nothing to do.
+//
+//   Y = RNbf16( X . W^T  +  RNbf16(s.T) . L2 ),   T = X . L1
+//
+// nlp-lineage "QLoRA" milestone page, section "The idea": the layer equation
+// (the 4-bit weight is dequantised to bf16 and multiplied, the adapters stay
+// bf16).  Three kernels, chained with programmatic dependent launch so each
+// one's launch overlaps the previous one's run:
+//
+// * lora_t_partial_kernel: T = X.L1 in K slices on CUDA cores (fp32).
+// * nf4_gemv_kernel: one CTA per SM holding three independent stream-K
+//   workers.  The work is the list of units (128-row tile of W, 256-wide k
+//   range) in row-tile-major order, cut into equal contiguous runs, one per
+//   worker, so every SM streams the same number of weight bytes whatever the
+//   shape.  A worker is four warps with a two-stage TMA ring (16 KB code tile
+//   of 128-byte rows + 8 KB X tile of 16 tokens, rows beyond M zero-filled).
+//   Each warp owns 32 rows of the tile and multiplies them with warp-level
+//   tensor-core MMAs (m16n8k16, bf16 in, fp32 accumulate in registers):
+//   the dequantised weights are produced directly as A fragments, so they
+//   never go through shared or tensor memory, and a segment's partial (a
+//   maximal run inside one row tile) is written straight from registers.
+//   Single-thread tcgen05 MMAs were measured to be the bottleneck here: with
+//   N = 16 each UMMA carries 128 x 16 weights and costs about as much to
+//   issue as a 128 x 256 one.
+//   The k order inside each 64-wide block is permuted identically in A and
+//   B (a sum is order-free up to rounding, and both operands see the same
+//   permutation): thread (g, c) of the warp takes code bytes 8c .. 8c+7 of
+//   its rows, i.e. k = 16c .. 16c+15, handing k-step s the pairs 2s (A
+//   columns 2c, 2c+1) and 2s+1 (columns 2c+8, 2c+9), and reads the matching
+//   X values k = 16c+4s .. 16c+4s+3 as one 8-byte load.
+//   Dequantisation uses a 64 KB shared-memory table of code pairs: entry e
+//   (one code byte: element 2j in the low nibble, 2j+1 in the high one) holds
+//   the fp32 levels (q[e & 15], q[e >> 4]), replicated for the 32 lanes so a
+//   warp's 8-byte loads never collide in a bank.  Per code byte: one byte
+//   permute forms the address, one LDS.64 fetches both levels, one packed
+//   multiply by the block scale c^ gives RN32(q.c^) for both weights and one
+//   conversion rounds the pair to bf16, i.e. exactly
+//   RNbf16(RN32(q[code].c^)), the dequantised weight of the pages; that
+//   bf16 pair is one A-fragment register.
+//   Warp 0: lanes 0..2 are the three TMA producers; the last warp sums this
+//   CTA's share of the T partials.
+// * gemv_finish_kernel: per row, the row tile's segment partials in worker
+//   order (deterministic) plus the LoRA term, rounded to bf16.
+#include "common.cuh"
+#include "internal.h"
+
+namespace qnf4 {
+namespace {
+
+constexpr int kWG = 3;                     // workers (groups of 4 warps) per CTA
+constexpr int kUnitKB = 4;                 // 64-wide k blocks per unit
+constexpr int kCodeBytes = 16384;          // 128 rows x 128 bytes (256 codes)
+constexpr int kXBytes = 8192;              // 16 tokens x 256 bf16 (4 boxes of 64)
+constexpr int kStageBytes = kCodeBytes + kXBytes;
+// Warps: 0 producers, 1 .. 4*kWG workers, last: T reduction.
+constexpr int kWarpT = 1 + 4 * kWG;
+constexpr int kGThreads = 32 * (kWarpT + 1);  // 448
+constexpr int kTabBytes = 65536;           // 256 pairs x 32 lanes x 8 bytes
+constexpr int kBarBytes = 1024;
+// Shared window: two stages and the barriers, then (at the next 64 KB
+// boundary, so the table's address bits 16.. come from one register in the
+// byte permute) the pair table, then the other four stages.
+constexpr int kFrontStages = 2;
+constexpr uint32_t kFrontBytes = kFrontStages * kStageBytes + kBarBytes;
+// With the dynamic window starting below 15 KB (it starts at 0 or 1 KB), the
+// layout ends at 64 KB + 64 KB + 4 stages = 224 KB; the kernel checks the fit.
+constexpr uint32_t kGemvSmemMin = 65536 + kTabBytes + (2 * kWG - kFrontStages) * kStageBytes;
+static_assert(kFrontBytes <= 65536 - 15360, "front region must fit below the table");
+
+struct GemvSmem {
+  uint32_t base;  // stages 0 .. kFrontStages-1 (codes, then X)
+  uint8_t* raw;
+  uint32_t raw_addr;
+  uint64_t* bars;
+  volatile int* abort_flag;
+  uint32_t tab;
+  bool fits;
+};
+
+QDEV GemvSmem carve(uint8_t* raw_ptr, uint32_t smem_bytes) {
+  GemvSmem g;
+  const uint32_t raw = smem_u32(raw_ptr);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t bars = base + kFrontStages * kStageBytes;
+  const uint32_t tab = (bars + kBarBytes + 0xFFFFu) & ~0xFFFFu;
+  g.base = base;
+  const uint32_t end = tab + kTabBytes + (2 * kWG - kFrontStages) * kStageBytes;
+  g.fits = end - raw <= smem_bytes && tab <= 0x00FF0000u;
+  g.raw = raw_ptr;
+  g.raw_addr = raw;
+  g.bars = reinterpret_cast<uint64_t*>(raw_ptr + (bars - raw));
+  g.abort_flag = reinterpret_cast<volatile int*>(g.bars + 64);
+  g.tab = tab;
+  return g;
+}
+
+// Barriers of worker g: full[2] (TMA bytes), empty[2] (one arrival per warp).
+QDEV uint64_t* bar_full(const GemvSmem& s, int g, int j) { return s.bars + g * 4 + j; }
+QDEV uint64_t* bar_empty(const GemvSmem& s, int g, int j) { return s.bars + g * 4 + 2 + j; }
+// Shared-window address of ring stage st (0 .. 2*kWG-1).
+QDEV uint32_t stage_addr(const GemvSmem& s, int st) {
+  return st < kFrontStages ? s.base + (uint32_t)(st * kStageBytes)
+                           : s.tab + kTabBytes + (uint32_t)((st - kFrontStages) * kStageBytes);
+}
+
+// The worker whose run holds unit u (runs: [w*U/W, (w+1)*U/W)).
+__host__ __device__ __forceinline__ int worker_of(int64_t u, int64_t U, int W) {
+  return (int)(((u + 1) * (int64_t)W - 1) / U);
+}
+
+QDEV float2 lds_pair(uint32_t addr) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+QDEV uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+// bf16x2 of code byte k (0..3) of word w: RNbf16(RN32(q[lo].c^)) low half,
+// RNbf16(RN32(q[hi].c^)) high half.  lanereg = table address bits 16..23 in
+// byte 2, lane * 8 in byte 0.
+QDEV uint32_t pair_lookup(uint32_t w, int k, uint32_t lanereg, float2 cc) {
+  const uint32_t addr = __byte_perm(w, lanereg, 0x7604u | ((uint32_t)k << 4));
+  const float2 p = __fmul2_rn(lds_pair(addr), cc);
+  return pack_bf16x2(p.x, p.y);
+}
+
+QDEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+QDEV bool warp_wait_g(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status, int lane) {
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (ok) mbar_try_wait(smem_u32(bar), parity);
+  return ok != 0;
+}
+
+QDEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+QDEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Block scales of unit (rt, un) for one weight row of the tile: the four
+// E4M3 codes packed in one word, and the c1 of the first and the last k
+// block (four consecutive blocks cross at most one 256-block group).
+struct RowScales {
+  uint32_t c2;
+  float c1a, c1b;
+};
+QDEV RowScales load_row_scales(const GemvArgs& a, int rt, int un, int rl) {
+  RowScales s{0u, 0.0f, 0.0f};
+  const int64_t n = (int64_t)rt * 128 + rl;
+  if (n >= a.N) return s;
+  const int kb0 = un * kUnitKB;
+  const int64_t f0 = n * a.kbt + kb0;
+  const int nkb = min(kUnitKB, a.kbt - kb0);
+#pragma unroll
+  for (int q = 0; q < kUnitKB; ++q)
+    if (q < nkb) s.c2 |= (uint32_t)__ldg(a.c2 + f0 + q) << (8 * q);
+  s.c1a = __ldg(a.c1 + (f0 >> 8));
+  s.c1b = __ldg(a.c1 + ((f0 + nkb - 1) >> 8));
+  return s;
+}
+// c^ of k block q (0..3) of the unit whose first block is f0's.
+QDEV float row_chat(const RowScales& s, int q, int64_t f0) {
+  const float c1 = ((f0 + q) >> 8) == (f0 >> 8) ? s.c1a : s.c1b;
+  return decode_scale((s.c2 >> (8 * q)) & 0xFFu, c1);
+}
+
+// NT = 8-token column tiles (1 for M <= 8, 2 for M <= 16).
+template <int NT>
+__global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_constant__ GemvArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const GemvSmem S = carve(smem_raw, args.smem_bytes);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (!S.fits) {  // shared-window layout not as planned: refuse, uniformly
+    if (tid == 0) report(args.status, QLORA_ERR_CUDA);
+    return;
+  }
+  const int G = gridDim.x, c = blockIdx.x;
+  const int W = G * kWG;
+  const int64_t U = args.units;
+  const int upr = args.upr;
+
+  if (tid == 0) {
+    for (int g = 0; g < kWG; ++g)
+      for (int j = 0; j < 2; ++j) {
+        mbar_init(bar_full(S, g, j), 1);
+        mbar_init(bar_empty(S, g, j), 4);
+      }
+    *S.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&args.tmCodes);
+    tma_prefetch_desc(&args.tmX);
+  }
+  // Pair table: entry e, lane l at tab + e*256 + l*8.
+  for (int idx = tid; idx < 256 * 32; idx += kGThreads) {
+    const int e = idx >> 5, l = idx & 31;
+    const float lo = args.q[e & 15], hi = args.q[e >> 4];
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(S.tab + (uint32_t)(e * 256 + l * 8)), "f"(lo), "f"(hi)
+                 : "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ----------------------------------------------- producers (lanes 0..2)
+    if (lane < kWG) {
+      const int g = lane, wk = c * kWG + g;
+      const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
+      const int nu = (int)(u1 - u0);
+      int issued = 0;
+      for (int i = 0; i < nu; ++i) {
+        const int j = i & 1;
+        if (!mbar_wait(bar_empty(S, g, j), ((uint32_t)(i >> 1) & 1u) ^ 1u, S.abort_flag, args.status)) break;
+        const int64_t u = u0 + i;
+        const int rt = (int)(u / upr), un = (int)(u % upr);
+        const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);  // k blocks of W in this unit
+        const uint32_t st = stage_addr(S, 2 * g + j);
+        uint8_t* sp = S.raw + (st - S.raw_addr);
+        mbar_arrive_expect_tx(bar_full(S, g, j), kCodeBytes + (uint32_t)nkb * 2048u);
+        tma_load_2d(sp, &args.tmCodes, bar_full(S, g, j), un * 128, rt * 128);
+        for (int q = 0; q < nkb; ++q)
+          tma_load_2d(sp + kCodeBytes + q * 2048, &args.tmX, bar_full(S, g, j), (un * kUnitKB + q) * 64, 0);
+        issued = i + 1;
+      }
+      if (*S.abort_flag) {  // let the loads already issued land before exit
+        for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
+          mbar_wait_drain(bar_full(S, g, i & 1), (uint32_t)(i >> 1) & 1u, 10000000ull);
+      }
+    }
+  } else if (warp == kWarpT) {
+    // ------------------------------------------------------ T reduction
+    // This CTA's share of T = sum_p Tp[p] (fixed order): T saved for the
+    // backward, RNbf16(s.T) for the finish kernel.  The T partials come from
+    // the previous kernel of the stream.
+    grid_dep_wait();
+    const int E = args.M * args.r, P = args.t_slices;
+    const int e_hi = (int)((int64_t)(c + 1) * E / G);
+    for (int e = (int)((int64_t)c * E / G) + lane; e < e_hi; e += 32) {
+      const int m = e / args.r, jj = e % args.r;
+      const float* src = args.tp + (int64_t)m * 128 + jj;
+      float T = 0.0f;
+      for (int p0 = 0; p0 < P; p0 += 8) {  // eight loads in flight, sum in slice order
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = p0 + k < P ? __ldg(src + (int64_t)(p0 + k) * 16 * 128) : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (p0 + k < P) T += v[k];
+      }
+      args.T_save[e] = T;
+      args.sTw[m * 128 + jj] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(args.s, T)));
+    }
+  } else {
+    // ------------------------------------------------- worker warps
+    const int g = (warp - 1) >> 2, wk = c * kWG + g, wq = (warp - 1) & 3;
+    const int gr = lane >> 2, cq = lane & 3;  // fragment row / column quad
+    // tile rows of this thread: two 16-row groups, rows gr and gr + 8 of each
+    int rows[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rows[i] = wq * 32 + (i >> 1) * 16 + (i & 1) * 8 + gr;
+    const uint32_t lanereg = (S.tab & 0x00FF0000u) | (uint32_t)(lane * 8);
+    const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
+    const int nu = (int)(u1 - u0);
+    float acc[2][NT][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[a][t][e] = 0.0f;
+    RowScales sc[4];
+    if (nu > 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sc[i] = load_row_scales(args, (int)(u0 / upr), (int)(u0 % upr), rows[i]);
+    }
+    bool aborted = false;
+    for (int i = 0; i < nu; ++i) {
+      const int64_t u = u0 + i;
+      const int rt = (int)(u / upr), un = (int)(u % upr);
+      const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);
+      const bool seg_end = i == nu - 1 || un == upr - 1;
+      RowScales cur[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) cur[r] = sc[r];
+      if (i + 1 < nu) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sc[r] = load_row_scales(args, (int)((u + 1) / upr), (int)((u + 1) % upr), rows[r]);
+      }
+      const int j = i & 1;
+      if (!aborted && !warp_wait_g(bar_full(S, g, j), (uint32_t)(i >> 1) & 1u, S.abort_flag, args.status, lane))
+        aborted = true;
+      if (!aborted) {
+        const uint32_t st = stage_addr(S, 2 * g + j);
+#pragma unroll
+        for (int q = 0; q < kUnitKB; ++q) {
+          if (q >= nkb) break;
+          // X fragments of the four k-steps: token n = 8t + gr, k = 16cq + 4s .. +3
+          uint2 xb[NT][4];
+          const uint32_t xt = st + kCodeBytes + (uint32_t)q * 2048;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const int n = 8 * t + gr;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+              xb[t][s] = lds64(xt + (uint32_t)n * 128 + ((((uint32_t)(2 * cq + (s >> 1))) ^ (uint32_t)(n & 7)) << 4) +
+                               8u * (uint32_t)(s & 1));
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // 16-row group h: rows[2h] (gr) and rows[2h+1] (gr + 8)
+            uint2 cw[2];
+            float2 cc[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int rl = rows[2 * h + e];
+              cw[e] = lds64(st + (uint32_t)rl * 128 +
+                            ((((uint32_t)(2 * q + (cq >> 1))) ^ (uint32_t)(rl & 7)) << 4) + 8u * (uint32_t)(cq & 1));
+              const int64_t f0 = ((int64_t)rt * 128 + rl) * args.kbt + (int64_t)un * kUnitKB;
+              const float ch = row_chat(cur[2 * h + e], q, f0);
+              cc[e] = make_float2(ch, ch);
+            }
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+              // code bytes 2s and 2s+1 of the thread's 8: word s >> 1, bytes 2(s&1), 2(s&1)+1
+              const uint32_t w0 = (s < 2) ? cw[0].x : cw[0].y;
+              const uint32_t w1 = (s < 2) ? cw[1].x : cw[1].y;
+              const int k0 = 2 * (s & 1);
+              const uint32_t a0 = pair_lookup(w0, k0, lanereg, cc[0]);
+              const uint32_t a1 = pair_lookup(w1, k0, lanereg, cc[1]);
+              const uint32_t a2 = pair_lookup(w0, k0 + 1, lanereg, cc[0]);
+              const uint32_t a3 = pair_lookup(w1, k0 + 1, lanereg, cc[1]);
+#pragma unroll
+              for (int t = 0; t < NT; ++t) mma_bf16_16816(acc[h][t], a0, a1, a2, a3, xb[t][s].x, xb[t][s].y);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty(S, g, j));  // this warp is done with the stage
+      if (seg_end) {
+        if (!aborted) {
+          const int jw = wk - worker_of((int64_t)rt * upr, U, W);
+          if (jw < 0 || jw >= args.maxc) {
+            if (lane == 0) report(args.status, QLORA_ERR_CUDA);
+          } else {
+            float* base = args.part + ((int64_t)rt * args.maxc + jw) * (16 * 128);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int m = 8 * t + 2 * cq + (e & 1);
+                  const int rl = rows[2 * h + (e >> 1)];
+                  if (m < args.M) base[m * 128 + rl] = acc[h][t][e];
+                }
+          }
+        }
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[a][t][e] = 0.0f;
+      }
+    }
+  }
+
+  __syncthreads();
+  grid_dep_launch();
+}
+
+// T partials: Tp[p][m][j] = sum over the k of slice p of X[m,k] L1[k,j], fp32,
+// fixed order, m < MB (M <= MB).  Slice p = k blocks [p*bps, (p+1)*bps),
+// walked in chunks of 256 rows staged in shared memory with every 16-byte
+// load of a chunk issued before the first use.  Thread t: column pair
+// jp = t % (r/2) and k lane kl = t / (r/2) (rows kl, kl + nkl, ...); the k
+// lanes' sums are added in lane order at the end.
+constexpr int kTChunk = 256;  // rows of L1 per staged chunk
+template <int MB>
+__global__ void __launch_bounds__(256) lora_t_partial_kernel(const uint16_t* __restrict__ X,
+                                                             const uint16_t* __restrict__ L1, int M, int64_t K,
+                                                             int r, int bps, float* __restrict__ tp) {
+  extern __shared__ __align__(16) uint8_t tsm[];
+  uint16_t* sL = reinterpret_cast<uint16_t*>(tsm);                    // [kTChunk][r]
+  uint16_t* sX = reinterpret_cast<uint16_t*>(tsm + kTChunk * r * 2);  // [16][kTChunk]
+  float* red = reinterpret_cast<float*>(tsm);                          // reused after the last chunk
+  grid_dep_launch();  // the GEMV kernel may start at once: it reads Tp only later
+  const int p = blockIdx.x, t = threadIdx.x;
+  const int64_t k_lo = (int64_t)p * bps * 64;
+  const int64_t k_hi = min((int64_t)(p + 1) * bps * 64, K);
+  const int r2 = r / 2, nkl = 256 / r2;
+  const int jp = t % r2, kl = t / r2;
+  float acc[MB][2];
+#pragma unroll
+  for (int i = 0; i < MB; ++i) acc[i][0] = acc[i][1] = 0.0f;
+  for (int64_t k0 = k_lo; k0 < k_hi; k0 += kTChunk) {
+    const int rows = (int)min((int64_t)kTChunk, k_hi - k0);  // a multiple of 64
+    const int nL = rows * r / 8, nX = M * rows / 8;            // 16-byte pieces
+    const uint4* gL = reinterpret_cast<const uint4*>(L1 + k0 * r);
+    for (int i = t; i < nL; i += 256) reinterpret_cast<uint4*>(sL)[i] = __ldg(gL + i);
+    for (int i = t; i < nX; i += 256) {
+      const int m = i / (rows / 8), cc = i % (rows / 8);
+      reinterpret_cast<uint4*>(sX + m * kTChunk)[cc] =
+          __ldg(reinterpret_cast<const uint4*>(X + (int64_t)m * K + k0) + cc);
+    }
+    __syncthreads();
+    if (kl < nkl) {
+      for (int k = kl; k < rows; k += nkl) {
+        const uint32_t lw = reinterpret_cast<const uint32_t*>(sL + k * r)[jp];
+        const float l0 = bf16_bits_to_float(lw & 0xFFFFu), l1 = bf16_bits_to_float(lw >> 16);
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          if (m < M) {
+            const float x = bf16_bits_to_float(sX[m * kTChunk + k]);
+            acc[m][0] = __fmaf_rn(x, l0, acc[m][0]);
+            acc[m][1] = __fmaf_rn(x, l1, acc[m][1]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // red[kl][m][j] (at most 256 x 32 floats: nkl * MB * r <= 256/r2 * 16 * 2 r2)
+  if (kl < nkl) {
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      red[(kl * MB + m) * r + 2 * jp] = acc[m][0];
+      red[(kl * MB + m) * r + 2 * jp + 1] = acc[m][1];
+    }
+  }
+  __syncthreads();
+  for (int idx = t; idx < M * r; idx += 256) {
+    const int m = idx / r, j = idx % r;
+    float sum = 0.0f;
+    for (int q = 0; q < nkl; ++q) sum += red[(q * MB + m) * r + j];
+    tp[((int64_t)p * 16 + m) * 128 + j] = sum;
+  }
+}
+
+// Y for 32 weight rows per CTA (128 threads), tokens m < MB (M <= MB).  Warp
+// w sums the row tile's partials of contributors j = w, w + 4, ... and the
+// LoRA products of adapter columns [w*r/4, (w+1)*r/4); the four warps' sums
+// are then added in warp order.
+template <int MB>
+__global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restrict__ part,
+                                                          const float* __restrict__ sTw,
+                                                          const uint16_t* __restrict__ L2, int M, int64_t N, int r,
+                                                          int upr, int64_t U, int W, int maxc,
+                                                          uint16_t* __restrict__ Y) {
+  __shared__ __align__(16) float sT[16 * 128];
+  __shared__ float red[4][MB][32];
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const int64_t n0 = (int64_t)blockIdx.x * 32, n = n0 + lane;
+  const int rt = (int)(n0 / 128), rl = (int)(n % 128);
+  const bool valid = n < N;
+  const int rq = r / 4, j0 = w * rq;  // this warp's adapter columns (r/4 is a multiple of 4)
+  // L2 first: it does not depend on the previous kernels
+  float l2v[32];
+#pragma unroll
+  for (int q = 0; q < 32; ++q)
+    l2v[q] = (valid && q < rq) ? bf16_bits_to_float(__ldg(L2 + (int64_t)(j0 + q) * N + n)) : 0.0f;
+  grid_dep_wait();
+  for (int idx = t; idx < M * 128; idx += 128) sT[idx] = sTw[idx];
+  const int c_lo = worker_of((int64_t)rt * upr, U, W);
+  const int cnt = min(worker_of((int64_t)(rt + 1) * upr - 1, U, W) - c_lo + 1, maxc);
+  float acc[MB];
+#pragma unroll
+  for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
+  for (int j = w; j < cnt; j += 4) {
+    const float* src = part + ((int64_t)rt * maxc + j) * (16 * 128) + rl;
+#pragma unroll
+    for (int m = 0; m < MB; ++m)
+      if (m < M) acc[m] += src[m * 128];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    if (q4 * 4 < rq) {
+#pragma unroll
+      for (int m = 0; m < MB; ++m) {
+        if (m < M) {
+          const float4 s4 = *reinterpret_cast<const float4*>(sT + m * 128 + j0 + q4 * 4);
+          acc[m] = __fmaf_rn(s4.x, l2v[q4 * 4 + 0], acc[m]);
+          acc[m] = __fmaf_rn(s4.y, l2v[q4 * 4 + 1], acc[m]);
+          acc[m] = __fmaf_rn(s4.z, l2v[q4 * 4 + 2], acc[m]);
+          acc[m] = __fmaf_rn(s4.w, l2v[q4 * 4 + 3], acc[m]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MB; ++m) red[w][m][lane] = acc[m];
+  __syncthreads();
+  if (w == 0 && valid) {
+#pragma unroll
+    for (int m = 0; m < MB; ++m)
+      if (m < M) {
+        const float y = ((red[0][m][lane] + red[1][m][lane]) + red[2][m][lane]) + red[3][m][lane];
+        reinterpret_cast<__nv_bfloat16*>(Y)[(int64_t)m * N + n] = __float2bfloat16_rn(y);
+      }
+  }
+}
+
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel of the stream still runs; it synchronises with
+// griddepcontrol.wait where it needs that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+}  // namespace
+
+GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int num_sms) {
+  (void)M;
+  GemvPlan p{};
+  p.m_tiles = (int)((N + 127) / 128);
+  p.kbt = (int)(K / 64);
+  p.upr = (p.kbt + kUnitKB - 1) / kUnitKB;
+  p.units = (int64_t)p.m_tiles * p.upr;
+  const int64_t want = (p.units + kWG - 1) / kWG;
+  p.grid = (int)(want < num_sms ? want : num_sms);
+  p.workers = p.grid * kWG;
+  const int64_t min_run = p.units / p.workers;  // 0 when some workers get nothing
+  p.maxc = min_run > 0 ? (int)((p.upr + min_run - 1) / min_run + 1) : p.workers;
+  if (p.maxc > p.workers) p.maxc = p.workers;
+  // T slices: at most kGemvTSlices, a whole number of k blocks each
+  p.bps = (p.kbt + kGemvTSlices - 1) / kGemvTSlices;
+  p.t_slices = (p.kbt + p.bps - 1) / p.bps;
+  p.part_bytes = (size_t)p.m_tiles * p.maxc * 16 * 128 * sizeof(float);
+  p.tp_bytes = (size_t)p.t_slices * 16 * 128 * sizeof(float);
+  p.stw_bytes = (size_t)16 * 128 * sizeof(float);
+  return p;
+}
+
+namespace {
+
+template <int MB>
+cudaError_t launch_gemv_mb(const GemvArgs& a, const GemvPlan& p, const uint16_t* X, const uint16_t* L1,
+                           const uint16_t* L2, uint16_t* Y, uint32_t smem, cudaStream_t st) {
+  // T kernel: staged chunk (L1 rows + X rows), reused for the k-lane sums
+  const int stage = kTChunk * a.r * 2 + 16 * kTChunk * 2;
+  const int tsmem = stage > 2048 * MB ? stage : 2048 * MB;
+  cudaError_t err = cudaFuncSetAttribute(lora_t_partial_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsmem);
+  if (err != cudaSuccess) return err;
+  GemvArgs args = a;
+  args.smem_bytes = smem;
+  args.t_slices = p.t_slices;
+  args.upr = p.upr;
+  lora_t_partial_kernel<MB><<<p.t_slices, 256, tsmem, st>>>(X, L1, a.M, a.K, a.r, p.bps, const_cast<float*>(a.tp));
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (a.M <= 8) err = launch_pdl(nf4_gemv_kernel<1>, dim3(p.grid), dim3(kGThreads), smem, st, args);
+  else err = launch_pdl(nf4_gemv_kernel<2>, dim3(p.grid), dim3(kGThreads), smem, st, args);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(gemv_finish_kernel<MB>, dim3((unsigned)((a.N + 31) / 32)), dim3(128), 0, st, a.part, a.sTw, L2,
+                   a.M, a.N, a.r, p.upr, p.units, p.workers, p.maxc, Y);
+  count_launches(3);
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& p, const uint16_t* X, const uint16_t* L1,
+                        const uint16_t* L2, uint16_t* Y, cudaStream_t st) {
+  int dev = 0, optin = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err == cudaSuccess) err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (err != cudaSuccess) return err;
+  if ((uint32_t)optin < kGemvSmemMin) return cudaErrorInvalidConfiguration;
+  const uint32_t smem = (uint32_t)optin;  // everything the block may have; the kernel checks its layout fits
+  err = cudaFuncSetAttribute(nf4_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(nf4_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  if (a.M <= 1) return launch_gemv_mb<1>(a, p, X, L1, L2, Y, smem, st);
+  if (a.M <= 4) return launch_gemv_mb<4>(a, p, X, L1, L2, Y, smem, st);
+  return launch_gemv_mb<16>(a, p, X, L1, L2, Y, smem, st);
+}
+
+}  // namespace qnf4

@@ -82,6 +82,57 @@ cudaError_t launch_engine(const EngineArgs& a, int amode, const GemmPlan& p, cud
 cudaError_t launch_split_reduce(const float* partial, int splits, int rows, int cols, const EpiArgs& e,
                                 cudaStream_t st);
 
+// ------------------------------------------------------------ small-M GEMV
+// Forward for M <= kGemvMaxM tokens: Y = X.W^T + s.(X.L1).L2 with the weight
+// streamed once from HBM.  Three kernels:
+//   (1) T partials: Tp[p][m][j] = sum_{k in slice p} X[m,k] L1[k,j]
+//   (2) stream-K dequant-GEMV: the units (128-row tile, 256-wide k range) of
+//       W split in equal runs over three workers per SM; every maximal run
+//       inside one row tile (a segment) leaves a 128 x 16 fp32 partial tile;
+//       one warp per CTA also sums its share of the T partials (T saved,
+//       RNbf16(s.T) for (3));
+//   (3) finish: Y = RNbf16(sum of a row tile's partials in worker order
+//       + RNbf16(s.T).L2).
+constexpr int kGemvMaxM = 16;
+constexpr int kGemvTSlices = 128;  // max T partial slices
+
+struct GemvPlan {
+  int m_tiles, kbt;   // 128-row tiles of W, 64-wide k blocks per row
+  int upr;            // units per row tile (256-wide k ranges)
+  int64_t units;      // m_tiles * upr
+  int grid, workers;  // CTAs (<= SMs), stream-K workers (3 per CTA)
+  int maxc;           // max workers covering one row tile
+  int t_slices, bps;  // T partial slices, k blocks per slice
+  size_t part_bytes;  // segment partials [m_tiles * maxc][16][128] fp32
+  size_t tp_bytes;    // T partials [t_slices][16][128] fp32
+  size_t stw_bytes;   // RNbf16(s.T) as fp32 [16][128]
+};
+
+struct GemvArgs {
+  CUtensorMap tmCodes;  // uint8 [N][K/2], box 128 x 128, 128-byte swizzle
+  CUtensorMap tmX;      // bf16 [M][K], box 64 x 16, 128-byte swizzle
+  const uint8_t* c2;
+  const float* c1;
+  int64_t N, K;
+  int M;
+  int kbt, upr, m_tiles, maxc;
+  int64_t units;
+  float* part;
+  // LoRA: T partials in, T (saved) and RNbf16(s.T) out
+  const float* tp;
+  int t_slices, r;
+  float s;
+  float* T_save;
+  float* sTw;
+  int* status;
+  uint32_t smem_bytes;
+  float q[16];
+};
+
+GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& p, const uint16_t* X, const uint16_t* L1,
+                        const uint16_t* L2, uint16_t* Y, cudaStream_t st);
+
 // --------------------------------------------------------- quantise kernels
 cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
                             int* status, cudaStream_t st);

@@ -83,6 +83,36 @@ def test_fwd_bwd_parity(lib, M, N, K, r, regime):
         assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} {regime}")
 
 
+# Few-token forward (M <= 16, the weight-streaming stream-K GEMV path): one
+# unit, ragged row tiles, a row tile spread over every CTA, CTAs with three
+# segments (K = 64), every T-slice thread layout (r = 48, 80, 128).
+GEMV_SHAPES = [
+    (1, 8, 64, 16), (7, 1000, 704, 32), (16, 2056, 1536, 48), (2, 128, 22016, 64),
+    (3, 40000, 64, 16), (16, 4096, 128, 128), (9, 384, 8192, 80), (12, 22016, 512, 64),
+]
+
+
+@pytest.mark.parametrize("M,N,K,r", GEMV_SHAPES)
+@pytest.mark.parametrize("regime", ["config", "lora_heavy"])
+def test_gemv_forward_parity(lib, M, N, K, r, regime):
+    s = 16.0 / r if regime == "config" else 0.75
+    case = make_case(M, N, K, r, seed=M * 13 + N + K + r, regime=regime)
+    got = run_gpu(lib, *case, s, backward=(regime == "config"))
+    ref = oracle_ref(*case, s, backward=(regime == "config"))
+    for k in got:
+        assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} {regime}")
+
+
+def test_gemv_forward_is_deterministic(lib):
+    X, W, L1, L2, _ = make_case(5, 2056, 2048, 64, seed=21)
+    tX, tW, tL1, tL2 = (from_bits(a) for a in (X, W, L1, L2))
+    w = lib.quantize(tW)
+    Y0, T0 = lib.linear_fwd(tX, w, tL1, tL2, 0.25)
+    Y1, T1 = lib.linear_fwd(tX, w, tL1, tL2, 0.25)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(Y0), bits(Y1)) and torch.equal(T0, T1)
+
+
 def test_zero_weight_is_pure_lora(lib):
     """W = 0: Y = s.X.L1.L2 and dX = s.dT.L1^T, so the LoRA extension is
     checked on its own."""
