@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqlora_nf4.so")
 SOURCES = ["api.cu", "engine.cu", "gemv.cu", "quant.cu", "noalloc.cu", "nf4_tables.cpp"]
-HEADERS = ["common.cuh", "internal.h"]
+HEADERS = ["common.cuh", "engine_util.cuh", "internal.h"]
 
 
 def nvcc_path() -> str:

@@ -19,17 +19,26 @@
 //
 // inferensys glossary "QLoRA", kernel paragraph: 4-bit weights are loaded,
 // decompressed in shared memory and fed to the tensor cores as BFloat16.
-#include "common.cuh"
-#include "internal.h"
+#include "engine_util.cuh"
 
 namespace qnf4 {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kDeqWarps = 16;                  // warps 2..17: dequant, then epilogue
-constexpr int kGroupWarps = 4;                 // one group of 4 warps per ring stage
-constexpr int kThreads = 64 + 32 * kDeqWarps;  // + producer warp + UMMA warp
-constexpr int kA = 16384;                      // 128 rows x 64 bf16
+constexpr int kGroupWarps = 4;  // a dequant group: 4 warps, one per TMEM lane quarter
+
+// Ring shape per A source.  The forward keeps its dequantised A tile in
+// TMEM, so its stages hold only B and the codes (36 KB) and six of them fit:
+// deep enough to cover the TMA latency plus the dequant of a stage at the
+// tensor-bound pace.  Three dequant groups (stage s always served by group
+// s % 3).  dX and the plain GEMMs keep A in shared memory: four 52 KB stages,
+// four groups.
+template <int AMODE>
+struct Ring {
+  static constexpr int S = AMODE == A_DEQ_K ? 6 : 4;     // stages
+  static constexpr int G = AMODE == A_DEQ_K ? 3 : 4;     // dequant (and epilogue) groups
+  static constexpr int KA = AMODE == A_DEQ_K ? 0 : 16384;  // A tile in shared memory (128 x 64 bf16)
+  static constexpr int THREADS = 64 + 32 * kGroupWarps * G;  // + producer warp + UMMA warp
+};
 
 // Tensor-memory columns: the fp32 accumulator (BN columns, at least 32) and,
 // for the forward fused GEMM, the dequantised A tile of every stage
@@ -38,64 +47,30 @@ template <int BN, int AMODE>
 struct Tmem {
   static constexpr uint32_t acc = BN < 32 ? 32 : BN;
   static constexpr uint32_t a_col = acc;
-  static constexpr uint32_t need = acc + (AMODE == A_DEQ_K ? kStages * 32 : 0);
+  static constexpr uint32_t need = acc + (AMODE == A_DEQ_K ? Ring<AMODE>::S * 32 : 0);
   static constexpr uint32_t cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 };
 
+// Stage = [A (KA)] [B] [codes].  In the forward the B slot also carries the
+// LoRA extension's A tiles (L2^T, 16 KB per 64-wide block, up to two), so it
+// is at least 32 KB there.
 template <int BN, int AMODE>
 struct Layout {
-  static constexpr int B = BN * 128 > 8192 ? BN * 128 : 8192;
+  static constexpr int BMIN = AMODE == A_DEQ_K ? 32768 : 8192;
+  static constexpr int B = BN * 128 > BMIN ? BN * 128 : BMIN;
   static constexpr int C = AMODE == A_TMA ? 0 : 4096;
-  static constexpr int STAGE = kA + B + C;
-  static constexpr int BAR = kStages * STAGE;
+  static constexpr int STAGE = Ring<AMODE>::KA + B + C;
+  static constexpr int BAR = Ring<AMODE>::S * STAGE;
   static constexpr int TOTAL = BAR + 256 + 1024;  // barriers etc. + alignment slack
 };
 
-QDEV uint32_t tx_bytes(int mn_major, int extent) {
-  return mn_major ? (uint32_t)((extent + 63) / 64) * 8192u : (uint32_t)extent * 128u;
-}
-
-// Load one operand tile (extent rows of UMMA M/N, 64 of the reduction).
-QDEV void load_operand(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int mn_major, int mn0, int k0,
-                       int extent) {
-  if (!mn_major) {
-    tma_load_2d(dst, m, bar, k0, mn0);
-  } else {
-    for (int j = 0; j < (extent + 63) / 64; ++j) tma_load_2d(dst + j * 8192, m, bar, mn0 + 64 * j, k0);
-  }
-}
-
-QDEV uint64_t operand_desc(const uint8_t* base, int mn_major, int kk) {
-  const uint32_t a = smem_u32(base);
-  return mn_major ? sdesc_sw128(a + kk * 2048, 8192, 1024) : sdesc_sw128(a + kk * 32, 16, 1024);
-}
-
-QDEV void epi_store(const EpiArgs& e, int64_t row, int64_t col, float v) {
-  if (e.out) {
-    const int64_t i = row * e.rs + col * e.cs;
-    if (e.out_bf16) reinterpret_cast<__nv_bfloat16*>(e.out)[i] = __float2bfloat16_rn(__fmul_rn(v, e.alpha));
-    else reinterpret_cast<float*>(e.out)[i] = __fmul_rn(v, e.alpha);
-  }
-  if (e.out2) {
-    const int64_t i = row * e.rs2 + col * e.cs2;
-    reinterpret_cast<__nv_bfloat16*>(e.out2)[i] = __float2bfloat16_rn(__fmul_rn(v, e.alpha2));
-  }
-}
-
-// Warp-wide wait: lane 0 polls (bounded), then every lane takes one
-// acquiring look at the completed phase.
-QDEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status, int lane) {
-  int ok = 1;
-  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
-  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  if (ok) mbar_try_wait(smem_u32(bar), parity);
-  return ok != 0;
-}
-
 template <int BN, int AMODE>
-__global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_constant__ EngineArgs args) {
+__global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(const __grid_constant__ EngineArgs args) {
   using L = Layout<BN, AMODE>;
   using TM = Tmem<BN, AMODE>;
+  using R = Ring<AMODE>;
+  constexpr int kStages = R::S;
+  constexpr int kA = R::KA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -110,7 +85,11 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
   const int kb_lo = (int)((int64_t)z * args.kb_main / args.splits);
   const int kb_hi = (int)((int64_t)(z + 1) * args.kb_main / args.splits);
   const int my_kb = kb_hi - kb_lo;
-  const int n_iters = my_kb + (z == 0 ? args.kb_ext : 0);
+  // The LoRA extension: forward = one stage with the L2^T tiles (A) then one
+  // stage per 64-wide block with the s.T tile (B); otherwise one stage per
+  // block holding both.
+  const int ext_iters = z == 0 && args.kb_ext ? (AMODE == A_DEQ_K ? 1 + args.kb_ext : args.kb_ext) : 0;
+  const int n_iters = my_kb + ext_iters;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -159,6 +138,16 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
           else if (AMODE == A_DEQ_MN) tma_load_2d(sc, &args.tmA, full + s, row0 / 2, kb * 64);
           else load_operand(sa, &args.tmA, full + s, args.a_mn_main, row0, kb * 64, 128);
           load_operand(sb, &args.tmB, full + s, args.b_mn_main, col0, kb * 64, BN);
+        } else if (AMODE == A_DEQ_K) {
+          if (it == my_kb) {  // all extension A tiles into this stage's B slot
+            mbar_arrive_expect_tx(full + s, (uint32_t)args.kb_ext * tx_bytes(args.a_mn_ext, 128));
+            for (int kb = 0; kb < args.kb_ext; ++kb)
+              load_operand(sb + kb * 16384, &args.tmAx, full + s, args.a_mn_ext, row0, kb * 64, 128);
+          } else {            // the s.T tile of extension block it - my_kb - 1
+            const int kb = it - my_kb - 1;
+            mbar_arrive_expect_tx(full + s, tx_bytes(args.b_mn_ext, BN));
+            load_operand(sb, &args.tmBx, full + s, args.b_mn_ext, col0, kb * 64, BN);
+          }
         } else {
           const int kb = it - my_kb;
           mbar_arrive_expect_tx(full + s, tx_bytes(args.a_mn_ext, 128) + tx_bytes(args.b_mn_ext, BN));
@@ -173,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
       const int a_mn_main = AMODE == A_DEQ_MN ? 1 : (AMODE == A_DEQ_K ? 0 : args.a_mn_main);
       const uint32_t id_main = idesc_bf16(128, BN, a_mn_main, args.b_mn_main);
       const uint32_t id_ext = idesc_bf16(128, BN, args.a_mn_ext, args.b_mn_ext);
+      int s_ext_a = -1;  // forward: stage holding the extension's A tiles
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -190,6 +180,20 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16_tmem_a(tmem_d, a_tmem + kk * 8, operand_desc(sb, args.b_mn_main, kk), id_main,
                              (it | kk) != 0);
+          umma_commit(empty + s);
+        } else if (AMODE == A_DEQ_K) {
+          if (it == my_kb) {  // the A tiles: keep the stage until the last extension block
+            s_ext_a = s;
+            continue;
+          }
+          const int kb = it - my_kb - 1;
+          const uint8_t* ea = smem + s_ext_a * L::STAGE + kA + kb * 16384;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_d, operand_desc(ea, args.a_mn_ext, kk), operand_desc(sb, args.b_mn_ext, kk), id_ext,
+                      (it | kk) != 0);
+          umma_commit(empty + s);
+          if (kb == args.kb_ext - 1) umma_commit(empty + s_ext_a);
         } else {
           const int amn = ext ? args.a_mn_ext : a_mn_main;
           const int bmn = ext ? args.b_mn_ext : args.b_mn_main;
@@ -197,33 +201,32 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tmem_d, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (it | kk) != 0);
+          umma_commit(empty + s);
         }
-        umma_commit(empty + s);
       }
       umma_commit(accum);
       committed_accum = true;
     }
     __syncwarp();
   } else {
-    const int dw = warp - 2;           // dequant warp 0..15
+    const int dw = warp - 2;           // dequant warp 0 .. 4G-1
     const int q4 = warp & 3;           // TMEM lane quarter this warp may access
-    const int grp = dw >> 2;           // group = the ring stage these 4 warps fill
+    const int grp = dw >> 2;           // group: iterations grp, grp + G, ...
     const int64_t bpr = args.wK / 64;  // NF4 blocks per weight row
     float q[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) q[i] = args.q[i];
     // ------------------------------------------------------------- dequant
-    // Group grp handles the iterations it = grp, grp + 4, ... (all in ring
-    // stage s = grp); each thread turns one whole NF4 block (64 weights,
-    // one scale) into bf16 per iteration.
+    // Group grp handles the iterations it = grp, grp + G, ... (ring stages
+    // it % S, always this group's since G divides S); each thread turns one
+    // whole NF4 block (64 weights, one scale) into bf16 per iteration.
     if (AMODE == A_DEQ_K) {
       // Thread: tile row rl (= TMEM lane), k = 0..63 of the stage.
       const int rl = q4 * 32 + lane;
       const int64_t n = row0 + rl;
       const bool valid = n < args.wN;
-      const uint32_t taddr = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col + (uint32_t)(grp * 32);
+      const uint32_t tlane = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col;
       const int sw = (rl >> 2) & 1;  // 32-byte swizzle of the code tile
-      const uint8_t* ctile = smem + grp * L::STAGE + kA + L::B + rl * 32;
       uint32_t c2raw = 0;
       float c1v = 0.0f;
       if (valid && grp < my_kb) {
@@ -231,18 +234,21 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
         c2raw = __ldg(args.c2 + f);
         c1v = __ldg(args.c1 + (f >> 8));
       }
-      for (int it = grp; it < my_kb; it += kStages) {
+      for (int it = grp; it < my_kb; it += R::G) {
+        const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        const uint32_t taddr = tlane + (uint32_t)(s * 32);
+        const uint8_t* ctile = smem + s * L::STAGE + kA + L::B + rl * 32;
         const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
-        if (valid && it + kStages < my_kb) {  // this group's next scale, one round ahead
-          const int64_t f = n * bpr + kb_lo + it + kStages;
+        if (valid && it + R::G < my_kb) {  // this group's next scale, one round ahead
+          const int64_t f = n * bpr + kb_lo + it + R::G;
           c2raw = __ldg(args.c2 + f);
           c1v = __ldg(args.c1 + (f >> 8));
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
-        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
+        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane)) break;
         tc_fence_after();
-        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
+        if (!warp_wait(full + s, ph, abort_flag, args.status, lane)) break;
         const uint4 c0 = *reinterpret_cast<const uint4*>(ctile + (sw << 4));
         const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + ((sw ^ 1) << 4));
         uint32_t o[16];
@@ -259,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(afull + grp);
+        if (lane == 0) mbar_arrive(afull + s);
       }
     } else if (AMODE == A_DEQ_MN) {
       // A = W^T in shared memory, MN-major: rows are k (W columns), the
@@ -320,15 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) umma_engine_kernel(const __grid_c
       }
     }
     // ------------------------------------------------------------ epilogue
-    // Four warps per lane quarter: group grp stores columns [grp*BN/4, ...).
+    // G warps per lane quarter: group grp stores the 16-column chunks
+    // grp, grp + G, ... of the tile.
     const bool ok = warp_wait(accum, 0, abort_flag, args.status, lane);
     tc_fence_after();
-    constexpr int kCols = BN >= 64 ? BN / 4 : 16;
-    const int c_lo = grp * kCols;
-    const int c_hi = c_lo + kCols < BN ? c_lo + kCols : BN;
     const int64_t row = row0 + q4 * 32 + lane;
     const EpiArgs& e = args.epi;
-    for (int c = c_lo; c < c_hi; c += 16) {
+    for (int c = grp * 16; c < BN; c += R::G * 16) {
       uint32_t v[16];
       tmem_ld16(tmem_d + ((uint32_t)(q4 * 32) << 16) + (uint32_t)c, v);
       tmem_wait_ld();
@@ -391,7 +395,7 @@ cudaError_t launch_t(const EngineArgs& a, const GemmPlan& p, cudaStream_t st) {
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
   if (err != cudaSuccess) return err;
   dim3 grid(p.m_tiles, p.n_tiles, p.splits);
-  kern<<<grid, kThreads, L::TOTAL, st>>>(a);
+  kern<<<grid, Ring<AMODE>::THREADS, L::TOTAL, st>>>(a);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -406,6 +410,17 @@ cudaError_t launch_mode(const EngineArgs& a, const GemmPlan& p, cudaStream_t st)
     case 256: return launch_t<256, AMODE>(a, p, st);
   }
   return cudaErrorInvalidValue;
+}
+
+template <int AMODE>
+size_t smem_for(int BN) {
+  switch (BN) {
+    case 16: return Layout<16, AMODE>::TOTAL;
+    case 32: return Layout<32, AMODE>::TOTAL;
+    case 64: return Layout<64, AMODE>::TOTAL;
+    case 128: return Layout<128, AMODE>::TOTAL;
+    default: return Layout<256, AMODE>::TOTAL;
+  }
 }
 
 }  // namespace
@@ -432,9 +447,11 @@ GemmPlan plan_gemm(int rows, int cols, int kb_main, int num_sms) {
 }
 
 size_t engine_smem_bytes(int BN, int amode) {
-  const int b = BN * 128 > 8192 ? BN * 128 : 8192;
-  const int c = amode == A_TMA ? 0 : 4096;
-  return (size_t)kStages * (kA + b + c) + 256 + 1024;
+  switch (amode) {
+    case A_DEQ_K: return smem_for<A_DEQ_K>(BN);
+    case A_DEQ_MN: return smem_for<A_DEQ_MN>(BN);
+    default: return smem_for<A_TMA>(BN);
+  }
 }
 
 cudaError_t launch_engine(const EngineArgs& a, int amode, const GemmPlan& p, cudaStream_t st) {
