@@ -41,6 +41,10 @@ sys.path.insert(0, ROOT)
 METRIC = ("fused QLoRA linear fwd+bwd TFLOP/s and % of roofline; "
           "NF4 (de)quant GB/s vs HBM peak")
 WORKLOAD = "llama7b_block"
+# DRAM bytes (read + write) per fused dequant-GEMM launch, averaged over the
+# 14 launches of a LLaMA-7B block step, from one ncu capture of the current
+# engine (profiles/fused_gemm_traffic_llama7b_block.md).
+FUSED_TRAFFIC_BYTES = 80.7e6
 RT_WORKLOAD = ("bulk NF4 round trip of 2^31 bf16 weights (4 GiB): half N(0, 0.02), half Student-t(3) x 0.02 "
                "with 0.1% outliers x50; one launch per direction")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -433,7 +437,8 @@ def run_ours(args):
             "e2e": {"value": e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "roofline": {"bound": "tensor", "kernel": "fused dequant-GEMM (Y forward, dX backward)",
                          "achieved": achieved, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops_sustained"], "traffic": None,
+                         "frac": achieved / pk["bf16_tflops_sustained"], "traffic": FUSED_TRAFFIC_BYTES,
+                         "traffic_unit": "bytes per launch (DRAM read + write, ncu, mean over the step's launches)",
                          "peak_source": f"{pk_kind} sustained dense bf16",
                          "launches_timed": 2 * n_lin, "ms_per_launch": gemm_ms / (2 * n_lin)},
             "quant": {"workload": RT_WORKLOAD, "value": quant_gbs, "unit": "GB/s", "frac": quant_gbs / hbm, "peak": hbm,
