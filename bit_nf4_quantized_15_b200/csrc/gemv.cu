@@ -49,14 +49,19 @@
 namespace qnf4 {
 namespace {
 
-constexpr int kWG = 3;                     // workers (groups of 4 warps) per CTA
+constexpr int kWG = 3;                     // stream-K workers per CTA
+constexpr int kWS = 2;                     // ring stages per worker
+constexpr int kNS = kWG * kWS;             // stages per CTA
 constexpr int kUnitKB = 4;                 // 64-wide k blocks per unit
 constexpr int kCodeBytes = 16384;          // 128 rows x 128 bytes (256 codes)
 constexpr int kXBytes = 8192;              // 16 tokens x 256 bf16 (4 boxes of 64)
 constexpr int kStageBytes = kCodeBytes + kXBytes;
-// Warps: 0 producers, 1 .. 4*kWG workers, last: T reduction.
-constexpr int kWarpT = 1 + 4 * kWG;
-constexpr int kGThreads = 32 * (kWarpT + 1);  // 448
+// A worker's warps each own kRG 16-row groups of the 128-row tile.
+constexpr int kRG = 2;
+constexpr int kWW = 8 / kRG;                  // warps per worker
+// Warps: 0 producers, 1 .. kWW*kWG workers, last: T reduction.
+constexpr int kWarpT = 1 + kWW * kWG;
+constexpr int kGThreads = 32 * (kWarpT + 1);
 constexpr int kTabBytes = 65536;           // 256 pairs x 32 lanes x 8 bytes
 constexpr int kBarBytes = 1024;
 // Shared window: two stages and the barriers, then (at the next 64 KB
@@ -66,7 +71,7 @@ constexpr int kFrontStages = 2;
 constexpr uint32_t kFrontBytes = kFrontStages * kStageBytes + kBarBytes;
 // With the dynamic window starting below 15 KB (it starts at 0 or 1 KB), the
 // layout ends at 64 KB + 64 KB + 4 stages = 224 KB; the kernel checks the fit.
-constexpr uint32_t kGemvSmemMin = 65536 + kTabBytes + (2 * kWG - kFrontStages) * kStageBytes;
+constexpr uint32_t kGemvSmemMin = 65536 + kTabBytes + (kNS - kFrontStages) * kStageBytes;
 static_assert(kFrontBytes <= 65536 - 15360, "front region must fit below the table");
 
 struct GemvSmem {
@@ -86,7 +91,7 @@ QDEV GemvSmem carve(uint8_t* raw_ptr, uint32_t smem_bytes) {
   const uint32_t bars = base + kFrontStages * kStageBytes;
   const uint32_t tab = (bars + kBarBytes + 0xFFFFu) & ~0xFFFFu;
   g.base = base;
-  const uint32_t end = tab + kTabBytes + (2 * kWG - kFrontStages) * kStageBytes;
+  const uint32_t end = tab + kTabBytes + (kNS - kFrontStages) * kStageBytes;
   g.fits = end - raw <= smem_bytes && tab <= 0x00FF0000u;
   g.raw = raw_ptr;
   g.raw_addr = raw;
@@ -96,10 +101,10 @@ QDEV GemvSmem carve(uint8_t* raw_ptr, uint32_t smem_bytes) {
   return g;
 }
 
-// Barriers of worker g: full[2] (TMA bytes), empty[2] (one arrival per warp).
-QDEV uint64_t* bar_full(const GemvSmem& s, int g, int j) { return s.bars + g * 4 + j; }
-QDEV uint64_t* bar_empty(const GemvSmem& s, int g, int j) { return s.bars + g * 4 + 2 + j; }
-// Shared-window address of ring stage st (0 .. 2*kWG-1).
+// Barriers of worker g: full[kWS] (TMA bytes), empty[kWS] (one arrival per warp).
+QDEV uint64_t* bar_full(const GemvSmem& s, int g, int j) { return s.bars + g * 2 * kWS + j; }
+QDEV uint64_t* bar_empty(const GemvSmem& s, int g, int j) { return s.bars + g * 2 * kWS + kWS + j; }
+// Shared-window address of ring stage st (0 .. kNS-1).
 QDEV uint32_t stage_addr(const GemvSmem& s, int st) {
   return st < kFrontStages ? s.base + (uint32_t)(st * kStageBytes)
                            : s.tab + kTabBytes + (uint32_t)((st - kFrontStages) * kStageBytes);
@@ -194,9 +199,9 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
 
   if (tid == 0) {
     for (int g = 0; g < kWG; ++g)
-      for (int j = 0; j < 2; ++j) {
+      for (int j = 0; j < kWS; ++j) {
         mbar_init(bar_full(S, g, j), 1);
-        mbar_init(bar_empty(S, g, j), 4);
+        mbar_init(bar_empty(S, g, j), kWW);
       }
     *S.abort_flag = 0;
     fence_mbar_init();
@@ -222,12 +227,12 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
       const int nu = (int)(u1 - u0);
       int issued = 0;
       for (int i = 0; i < nu; ++i) {
-        const int j = i & 1;
-        if (!mbar_wait(bar_empty(S, g, j), ((uint32_t)(i >> 1) & 1u) ^ 1u, S.abort_flag, args.status)) break;
+        const int j = i % kWS;
+        if (!mbar_wait(bar_empty(S, g, j), ((uint32_t)(i / kWS) & 1u) ^ 1u, S.abort_flag, args.status)) break;
         const int64_t u = u0 + i;
         const int rt = (int)(u / upr), un = (int)(u % upr);
         const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);  // k blocks of W in this unit
-        const uint32_t st = stage_addr(S, 2 * g + j);
+        const uint32_t st = stage_addr(S, kWS * g + j);
         uint8_t* sp = S.raw + (st - S.raw_addr);
         mbar_arrive_expect_tx(bar_full(S, g, j), kCodeBytes + (uint32_t)nkb * 2048u);
         tma_load_2d(sp, &args.tmCodes, bar_full(S, g, j), un * 128, rt * 128);
@@ -236,8 +241,8 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
         issued = i + 1;
       }
       if (*S.abort_flag) {  // let the loads already issued land before exit
-        for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
-          mbar_wait_drain(bar_full(S, g, i & 1), (uint32_t)(i >> 1) & 1u, 10000000ull);
+        for (int i = issued - kWS > 0 ? issued - kWS : 0; i < issued; ++i)
+          mbar_wait_drain(bar_full(S, g, i % kWS), (uint32_t)(i / kWS) & 1u, 10000000ull);
       }
     }
   } else if (warp == kWarpT) {
@@ -265,26 +270,26 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------- worker warps
-    const int g = (warp - 1) >> 2, wk = c * kWG + g, wq = (warp - 1) & 3;
+    const int g = (warp - 1) / kWW, wk = c * kWG + g, wq = (warp - 1) % kWW;
     const int gr = lane >> 2, cq = lane & 3;  // fragment row / column quad
-    // tile rows of this thread: two 16-row groups, rows gr and gr + 8 of each
-    int rows[4];
+    // tile rows of this thread: kRG 16-row groups, rows gr and gr + 8 of each
+    int rows[2 * kRG];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) rows[i] = wq * 32 + (i >> 1) * 16 + (i & 1) * 8 + gr;
+    for (int i = 0; i < 2 * kRG; ++i) rows[i] = wq * 16 * kRG + (i >> 1) * 16 + (i & 1) * 8 + gr;
     const uint32_t lanereg = (S.tab & 0x00FF0000u) | (uint32_t)(lane * 8);
     const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
     const int nu = (int)(u1 - u0);
-    float acc[2][NT][4];
+    float acc[kRG][NT][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int a = 0; a < kRG; ++a)
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[a][t][e] = 0.0f;
-    RowScales sc[4];
+    RowScales sc[2 * kRG];
     if (nu > 0) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sc[i] = load_row_scales(args, (int)(u0 / upr), (int)(u0 % upr), rows[i]);
+      for (int i = 0; i < 2 * kRG; ++i) sc[i] = load_row_scales(args, (int)(u0 / upr), (int)(u0 % upr), rows[i]);
     }
     bool aborted = false;
     for (int i = 0; i < nu; ++i) {
@@ -292,18 +297,18 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
       const int rt = (int)(u / upr), un = (int)(u % upr);
       const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);
       const bool seg_end = i == nu - 1 || un == upr - 1;
-      RowScales cur[4];
+      RowScales cur[2 * kRG];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) cur[r] = sc[r];
+      for (int r = 0; r < 2 * kRG; ++r) cur[r] = sc[r];
       if (i + 1 < nu) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) sc[r] = load_row_scales(args, (int)((u + 1) / upr), (int)((u + 1) % upr), rows[r]);
+        for (int r = 0; r < 2 * kRG; ++r) sc[r] = load_row_scales(args, (int)((u + 1) / upr), (int)((u + 1) % upr), rows[r]);
       }
-      const int j = i & 1;
-      if (!aborted && !warp_wait_g(bar_full(S, g, j), (uint32_t)(i >> 1) & 1u, S.abort_flag, args.status, lane))
+      const int j = i % kWS;
+      if (!aborted && !warp_wait_g(bar_full(S, g, j), (uint32_t)(i / kWS) & 1u, S.abort_flag, args.status, lane))
         aborted = true;
       if (!aborted) {
-        const uint32_t st = stage_addr(S, 2 * g + j);
+        const uint32_t st = stage_addr(S, kWS * g + j);
 #pragma unroll
         for (int q = 0; q < kUnitKB; ++q) {
           if (q >= nkb) break;
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
                                8u * (uint32_t)(s & 1));
           }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {  // 16-row group h: rows[2h] (gr) and rows[2h+1] (gr + 8)
+          for (int h = 0; h < kRG; ++h) {  // 16-row group h: rows[2h] (gr) and rows[2h+1] (gr + 8)
             uint2 cw[2];
             float2 cc[2];
 #pragma unroll
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
           } else {
             float* base = args.part + ((int64_t)rt * args.maxc + jw) * (16 * 128);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < kRG; ++h)
 #pragma unroll
               for (int t = 0; t < NT; ++t)
 #pragma unroll
@@ -369,7 +374,7 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
           }
         }
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
+        for (int a = 0; a < kRG; ++a)
 #pragma unroll
           for (int t = 0; t < NT; ++t)
 #pragma unroll
