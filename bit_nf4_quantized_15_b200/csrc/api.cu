@@ -3,6 +3,7 @@
 // synchronisation: all work is queued on the caller's stream.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -105,10 +106,24 @@ void fill_common(EngineArgs* a, int* status) {
   for (int i = 0; i < 16; ++i) a->q[i] = t.q[i];
 }
 
+// The forward dequant-GEMM on CTA pairs (launch_pair_fwd): used, for plans
+// with full 256-token tiles and no split, when QLORA_NF4_PAIR=1 is set in
+// the environment.  It computes the same result as the single-CTA engine
+// and measured slower on the LLaMA-7B linears, so the single-CTA engine is
+// the default.
+constexpr int A_PAIR_K = 3;
+
+bool use_pair_fwd(const GemmPlan& p, int rows, int cols, int kb_ext) {
+  if (p.BN != 256 || p.splits != 1 || !pair_fwd_supported(rows, cols, kb_ext)) return false;
+  const char* env = std::getenv("QLORA_NF4_PAIR");
+  return env && env[0] == '1';
+}
+
 // Launch the engine and, for a split reduction, the fixed-order sum.
 int run(EngineArgs& a, int amode, const GemmPlan& p, float* partial, cudaStream_t st) {
   a.splits = p.splits;
   a.partial = p.splits > 1 ? partial : nullptr;
+  if (amode == A_PAIR_K) return launch_pair_fwd(a, st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
   if (launch_engine(a, amode, p, st) != cudaSuccess) return QLORA_ERR_CUDA;
   if (p.splits > 1 && launch_split_reduce(partial, p.splits, a.rows, a.cols, a.epi, st) != cudaSuccess)
     return QLORA_ERR_CUDA;
@@ -328,9 +343,13 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
     EngineArgs a;
     fill_common(&a, status_dev);
     const GemmPlan& p = lay.y_fwd;
-    if (map_codes(&a.tmA, w->codes, N, K, 0) || map_operand(&a.tmB, X, 0, M, K, p.BN) ||
-        map_operand(&a.tmAx, L2, 1, N, r, 128) || map_operand(&a.tmBx, sT, 0, M, r, p.BN))
+    const int kb_ext = (r + 63) / 64;
+    const bool pair = use_pair_fwd(p, (int)N, (int)M, kb_ext);
+    const int brows = pair ? 128 : p.BN;  // a pair CTA holds half of the 256 tokens
+    if (map_codes(&a.tmA, w->codes, N, K, 0) || map_operand(&a.tmB, X, 0, M, K, brows) ||
+        map_operand(&a.tmAx, L2, 1, N, r, 128) || map_operand(&a.tmBx, sT, 0, M, r, brows))
       return QLORA_ERR_CUDA;
+    a.codes = w->codes;
     a.c2 = w->c2;
     a.c1 = w->c1;
     a.wN = N;
@@ -338,14 +357,14 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
     a.rows = (int)N;
     a.cols = (int)M;
     a.kb_main = (int)(K / 64);
-    a.kb_ext = (r + 63) / 64;
+    a.kb_ext = kb_ext;
     a.a_mn_ext = 1;
     a.epi = epi_none();
     a.epi.out = Y;
     a.epi.out_bf16 = 1;
     a.epi.rs = 1;
     a.epi.cs = N;
-    if (int rc = run_timed(a, A_DEQ_K, p, partial, st)) return rc;
+    if (int rc = run_timed(a, pair ? A_PAIR_K : A_DEQ_K, p, partial, st)) return rc;
   }
   return QLORA_OK;
 }

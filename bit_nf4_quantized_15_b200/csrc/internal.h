@@ -56,6 +56,7 @@ struct EngineArgs {
   CUtensorMap tmB;   // main B
   CUtensorMap tmAx;  // extension A (LoRA term)
   CUtensorMap tmBx;  // extension B
+  const uint8_t* codes;  // NF4 codes [wN][wK/2] (read directly by the pair forward)
   const uint8_t* c2;
   const float* c1;
   int64_t wN, wK;    // quantised weight shape (for scale indexing)
@@ -81,6 +82,14 @@ size_t engine_smem_bytes(int BN, int amode);
 cudaError_t launch_engine(const EngineArgs& a, int amode, const GemmPlan& p, cudaStream_t st);
 cudaError_t launch_split_reduce(const float* partial, int splits, int rows, int cols, const EpiArgs& e,
                                 cudaStream_t st);
+
+// Forward dequant-GEMM on CTA pairs (cta_group::2, 256 x 256 output tile per
+// pair).  Same EngineArgs as A_DEQ_K with these tensor maps: tmA codes (box
+// 32 x 128 bytes), tmB X (K-major, box 64 x 128), tmAx L2 (MN-major, 64 x 64),
+// tmBx RNbf16(s.T) (K-major, box 64 x 128); bf16 output, no split.
+bool pair_fwd_supported(int rows, int cols, int kb_ext);
+size_t pair_fwd_smem_bytes();
+cudaError_t launch_pair_fwd(const EngineArgs& a, cudaStream_t st);
 
 // ------------------------------------------------------------ small-M GEMV
 // Forward for M <= kGemvMaxM tokens: Y = X.W^T + s.(X.L1).L2 with the weight

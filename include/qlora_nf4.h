@@ -130,6 +130,9 @@ QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  *   Y   : bf16[M][N]     T_save : float[M][r]
  *   ws  : device workspace of ws_bytes >= qlora_workspace_bytes(M, N, K, r)
  * Requires K % 64 == 0, N % 8 == 0, r % 16 == 0 and 16 <= r <= 128.
+ * With QLORA_NF4_PAIR=1 in the environment (read at each call), grids of at
+ * least one 128 x 256 tile per SM run on the CTA-pair kernel (cta_group::2)
+ * instead of the single-CTA one: same result within the same tolerance.
  */
 QLORA_API int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
                      const uint16_t* L1, const uint16_t* L2, int r, float s, uint16_t* Y,

@@ -83,6 +83,28 @@ def test_fwd_bwd_parity(lib, M, N, K, r, regime):
         assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} {regime}")
 
 
+# Forward on CTA pairs (256 x 256 output tile per pair of SMs): grids with at
+# least one tile per SM and 256-token tiles.  The last pair's odd CTA entirely
+# beyond N (4736 = 18.5 x 256), ragged tokens inside the odd CTA's half
+# (1000) or the even one's (1800), two LoRA extension blocks (r = 128) and
+# fewer k-blocks than dequant groups (K = 192), r = 16 zero-filled to 64.
+# The pair path is opt-in (QLORA_NF4_PAIR=1); each case also runs on the
+# default single-CTA engine.
+PAIR_SHAPES = [(1000, 4736, 256, 64), (1800, 4000, 192, 128), (600, 9000, 128, 16), (2048, 4096, 512, 32)]
+
+
+@pytest.mark.parametrize("M,N,K,r", PAIR_SHAPES)
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_pair_forward_parity(lib, monkeypatch, M, N, K, r, pair):
+    monkeypatch.setenv("QLORA_NF4_PAIR", pair)
+    s = 0.75
+    case = make_case(M, N, K, r, seed=M * 11 + N + K + r, regime="lora_heavy")
+    got = run_gpu(lib, *case, s, backward=False)
+    ref = oracle_ref(*case, s, backward=False)
+    for k in got:
+        assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} pair={pair}")
+
+
 # Few-token forward (M <= 16, the weight-streaming stream-K GEMV path): one
 # unit, ragged row tiles, a row tile spread over every CTA, CTAs with three
 # segments (K = 64), every T-slice thread layout (r = 48, 80, 128).
