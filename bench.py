@@ -367,28 +367,39 @@ def run_ours(args):
     rt_n = WL.ROUNDTRIP_WEIGHTS
     rt_N, rt_K = rt_n // 4096, 4096
     Wrt = WL.roundtrip_weights(rt_n, seed=0, device=dev).view(rt_N, rt_K)
-    wrt = q.NF4Weight.empty(rt_N, rt_K, dev)
     Wout = torch.empty_like(Wrt)
     qb, db = quant_bytes(rt_N, rt_K), dequant_bytes(rt_N, rt_K)
-    for _ in range(2):
-        q.quantize_into(Wrt, wrt)
-        q.dequant(wrt, out=Wout)
-    torch.cuda.synchronize()
     reps = max(args.steps, 3)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    for _ in range(reps):
-        q.quantize_into(Wrt, wrt)
-    a1.record()
-    torch.cuda.synchronize()
-    quant_gbs = qb * reps / (a0.elapsed_time(a1) / 1e3) / 1e9
-    a0.record()
-    for _ in range(reps):
-        q.dequant(wrt, out=Wout)
-    a1.record()
-    torch.cuda.synchronize()
-    dequant_gbs = db * reps / (a0.elapsed_time(a1) / 1e3) / 1e9
-    del Wrt, wrt, Wout
+
+    def roundtrip(fmt):
+        """(quantise GB/s, dequantise GB/s) of one format on the round trip."""
+        wrt = q.NF4Weight.empty(rt_N, rt_K, dev, fmt)
+        for _ in range(2):
+            q.quantize_into(Wrt, wrt)
+            q.dequant(wrt, out=Wout)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(reps):
+            q.quantize_into(Wrt, wrt)
+        a1.record()
+        torch.cuda.synchronize()
+        qg = qb * reps / (a0.elapsed_time(a1) / 1e3) / 1e9
+        a0.record()
+        for _ in range(reps):
+            q.dequant(wrt, out=Wout)
+        a1.record()
+        torch.cuda.synchronize()
+        return qg, db * reps / (a0.elapsed_time(a1) / 1e3) / 1e9
+
+    quant_gbs, dequant_gbs = roundtrip("nf4")
+    # the two 4-bit formats the method is compared with (same round trip)
+    formats = {}
+    for fmt in ("fp4", "int4"):
+        qg, dg = roundtrip(fmt)
+        formats[fmt] = {"quant_gbs": qg, "quant_frac": qg / pk["hbm_gbs"], "dequant_gbs": dg,
+                        "dequant_frac": dg / pk["hbm_gbs"]}
+    del Wrt, Wout
     assert q.read_status(dev) == 0
 
     # ---- few-token forward (dequant-GEMV regime): LLaMA-65B FFN up and down
@@ -445,6 +456,8 @@ def run_ours(args):
                       "bytes": qb, "peak_source": f"{pk_kind} HBM copy"},
             "dequant": {"workload": RT_WORKLOAD, "value": dequant_gbs, "unit": "GB/s", "frac": dequant_gbs / hbm, "peak": hbm,
                         "bytes": db, "peak_source": f"{pk_kind} HBM copy"},
+            "formats": {"workload": RT_WORKLOAD + "; FP4 = E2M1/6 and Int4 = k/7 levels (the compared formats)",
+                        "unit": "GB/s", **formats},
             "gemv": gemv,
             "cpu_baseline": base,
             "clocks": clk,

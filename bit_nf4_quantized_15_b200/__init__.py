@@ -6,7 +6,7 @@ computation runs in the library's CUDA kernels.  PyTorch is used for device
 memory and the current stream.  There is no CPU fallback: if the library
 is missing or the device is not sm_100, calls raise.
 
-    w = quantize(W)                       # NF4 double quantisation
+    w = quantize(W)                       # NF4 double quantisation (fmt="fp4"/"int4": compared formats)
     What = dequant(w)                     # doubleDequant -> bf16
     Y, T = linear_fwd(X, w, L1, L2, s)    # Y = X.W^T + s.X.L1.L2
     dX, dL1, dL2 = linear_bwd(dY, X, T, w, L1, L2, s)
@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "lib", "NF4Weight", "quantize", "quantize_into", "dequant", "workspace_bytes", "linear_fwd", "linear_bwd",
-    "codebook", "status_string", "kernel_launches", "set_gemm_events", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
+    "codebook", "FORMATS", "status_string", "kernel_launches", "set_gemm_events", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
@@ -31,6 +31,10 @@ QLORA_OK = 0
 QLORA_ERR_NONFINITE = -7
 QLORA_ERR_TIMEOUT = -8
 
+# Code formats (QLORA_FMT_*): NF4, and the two 4-bit formats the method is
+# compared with (FP4 = E2M1/6, Int4 = k/7).
+FORMATS = {"nf4": 0, "fp4": 1, "int4": 2}
+
 
 class QLoRAError(RuntimeError):
     pass
@@ -38,7 +42,8 @@ class QLoRAError(RuntimeError):
 
 class qlora_nf4_weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p),
-                ("n_rows", ctypes.c_int64), ("n_cols", ctypes.c_int64)]
+                ("n_rows", ctypes.c_int64), ("n_cols", ctypes.c_int64),
+                ("format", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _lib = None
@@ -49,6 +54,7 @@ _SIGS = {
     "qlora_nf4_storage_bytes": (ctypes.c_int, [_I64, _I64, ctypes.POINTER(ctypes.c_size_t),
                                                ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
     "qlora_nf4_codebook": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float)]),
+    "qlora_code_levels": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_float)]),
     "qlora_nf4_quantize": (ctypes.c_int, [_P, _I64, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P]),
     "qlora_nf4_dequant": (ctypes.c_int, [ctypes.POINTER(qlora_nf4_weight), _P, _P, _P]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int]),
@@ -147,31 +153,39 @@ def storage_bytes(N: int, K: int):
 
 @dataclass
 class NF4Weight:
-    """Quantized weight: codes uint8[N*K/2], c2 uint8[N*K/64] (E4M3), c1 float32[ceil(N*K/16384)]."""
+    """Quantized weight: codes uint8[N*K/2], c2 uint8[N*K/64] (E4M3), c1 float32[ceil(N*K/16384)];
+    ``fmt`` names the 16 levels the codes index (see FORMATS)."""
     codes: torch.Tensor
     c2: torch.Tensor
     c1: torch.Tensor
     N: int
     K: int
+    fmt: str = "nf4"
 
     def descriptor(self) -> qlora_nf4_weight:
-        return qlora_nf4_weight(self.codes.data_ptr(), self.c2.data_ptr(), self.c1.data_ptr(), self.N, self.K)
+        if self.fmt not in FORMATS:
+            raise QLoRAError(f"unknown format {self.fmt!r}")
+        return qlora_nf4_weight(self.codes.data_ptr(), self.c2.data_ptr(), self.c1.data_ptr(), self.N, self.K,
+                                FORMATS[self.fmt], 0)
 
     @property
     def device(self):
         return self.codes.device
 
     @staticmethod
-    def empty(N: int, K: int, device="cuda") -> "NF4Weight":
+    def empty(N: int, K: int, device="cuda", fmt: str = "nf4") -> "NF4Weight":
         nc, n2, n1 = storage_bytes(N, K)
         return NF4Weight(torch.empty(nc, dtype=torch.uint8, device=device),
                          torch.empty(n2, dtype=torch.uint8, device=device),
-                         torch.empty(n1 // 4, dtype=torch.float32, device=device), N, K)
+                         torch.empty(n1 // 4, dtype=torch.float32, device=device), N, K, fmt)
 
 
-def codebook():
+def codebook(fmt: str = "nf4"):
+    """The 16 ascending levels the kernels use for a format."""
+    if fmt not in FORMATS:
+        raise QLoRAError(f"unknown format {fmt!r}")
     arr = (ctypes.c_float * 16)()
-    _check(lib().qlora_nf4_codebook(arr))
+    _check(lib().qlora_code_levels(FORMATS[fmt], arr))
     return [float(v) for v in arr]
 
 
@@ -184,11 +198,12 @@ def quantize_into(W: torch.Tensor, out: NF4Weight, status=None):
     return out
 
 
-def quantize(W: torch.Tensor, status=None) -> NF4Weight:
-    """NF4 double quantisation of a bf16 CUDA weight [N, K] (K % 64 == 0)."""
+def quantize(W: torch.Tensor, status=None, fmt: str = "nf4") -> NF4Weight:
+    """NF4 double quantisation of a bf16 CUDA weight [N, K] (K % 64 == 0);
+    fmt="fp4" or "int4" quantises to one of the compared formats instead."""
     _bf16_cuda(W, "W")
     N, K = W.shape
-    return quantize_into(W, NF4Weight.empty(N, K, W.device), status)
+    return quantize_into(W, NF4Weight.empty(N, K, W.device, fmt), status)
 
 
 def dequant(w: NF4Weight, out: torch.Tensor | None = None, status=None) -> torch.Tensor:

@@ -26,6 +26,14 @@ struct Nf4Tables {
 // Derived once per process on the host, from the normal quantiles.
 const Nf4Tables& nf4_tables();
 
+// Code formats (QLORA_FMT_*): NF4, and the two formats the method is
+// compared with, FP4 (E2M1 / 6) and Int4 (k / 7), each with a pad level
+// below -1 that is never produced.  Same table layout; only NF4 has a
+// code-search polynomial (poly_ok is false for the others, whose quantiser
+// searches the thresholds).
+constexpr int kNumFormats = 3;
+const Nf4Tables& code_tables(int format);  // format in [0, kNumFormats)
+
 // Process-wide count of kernels launched through the library.
 void count_launches(uint64_t n);
 uint64_t launches_so_far();
@@ -144,9 +152,9 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& p, const uint16_t* X,
 
 // --------------------------------------------------------- quantise kernels
 cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
-                            int* status, cudaStream_t st);
+                            int* status, int format, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
-                           uint16_t* out, cudaStream_t st);
+                           uint16_t* out, int format, cudaStream_t st);
 cudaError_t launch_scale_to_bf16(const float* in, int64_t n, float s, uint16_t* out, cudaStream_t st);
 
 }  // namespace qnf4

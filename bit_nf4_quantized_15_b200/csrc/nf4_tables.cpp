@@ -115,6 +115,37 @@ Nf4Tables build() {
   return t;
 }
 
+// Levels given as doubles (each the correctly rounded fp64 value of an exact
+// rational), rounded once to fp32, with their thresholds.
+Nf4Tables from_levels(const double (&lv)[16]) {
+  Nf4Tables t{};
+  for (int i = 0; i < 16; ++i) t.q[i] = (float)lv[i];
+  for (int i = 0; i < 15; ++i) t.t[i] = round_down_to_float(((double)t.q[i] + (double)t.q[i + 1]) * 0.5);
+  t.poly_ok = false;
+  return t;
+}
+
+// "A standard 4-bit float" (section "What it showed", third bullet): OCP
+// E2M1 magnitudes 0, 1/2, 1, 3/2, 2, 3, 4, 6 over 6, mirrored, one zero,
+// and the pad level -2.
+Nf4Tables build_fp4() {
+  const double mags[7] = {0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  double lv[16];
+  lv[0] = -2.0;
+  for (int i = 0; i < 7; ++i) lv[1 + i] = -mags[6 - i] / 6.0;
+  lv[8] = 0.0;
+  for (int i = 0; i < 7; ++i) lv[9 + i] = mags[i] / 6.0;
+  return from_levels(lv);
+}
+
+// "4-bit integers" (same bullet): symmetric levels k/7, k = -7 .. 7, and the
+// unused two's-complement code -8 as the pad level -8/7.
+Nf4Tables build_int4() {
+  double lv[16];
+  for (int k = -8; k < 8; ++k) lv[k + 8] = (double)k / 7.0;
+  return from_levels(lv);
+}
+
 }  // namespace
 
 namespace {
@@ -129,6 +160,16 @@ const Nf4Tables& nf4_tables() {
   static std::once_flag once;
   std::call_once(once, [] { tables = build(); });
   return tables;
+}
+
+const Nf4Tables& code_tables(int format) {
+  static Nf4Tables fp4, int4;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    fp4 = build_fp4();
+    int4 = build_int4();
+  });
+  return format == 1 ? fp4 : format == 2 ? int4 : nf4_tables();
 }
 
 }  // namespace qnf4

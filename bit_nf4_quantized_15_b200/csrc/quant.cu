@@ -1,5 +1,6 @@
 // NF4 double quantisation (bf16 -> codes, c2, c1) and dequantisation
-// (codes, c2, c1 -> bf16): the two HBM-bound passes.
+// (codes, c2, c1 -> bf16): the two HBM-bound passes.  The same kernels serve
+// the two compared 4-bit formats (FP4, Int4), which swap only the levels.
 //
 // nlp-lineage "QLoRA" milestone page, section "The idea": blocks of 64
 // weights with an absmax scale, the scales themselves quantised to 8 bits
@@ -67,8 +68,31 @@ QDEV uint32_t nf4_codes8(const float2 (&x)[4], const float2 (&P)[6], uint32_t t_
   return acc - kMagicBits * 0x11111111u;  // remove sum_i magic * 16^i (mod 2^32)
 }
 
+// Codes of four pairs x[0..3] for any 16-level table: a branch-free binary
+// search over the 15 thresholds (code = number of thresholds below x), the
+// thresholds read from shared memory (16 words in 16 banks: no conflicts).
+// Used for the compared formats, whose levels have no fitted polynomial.
+QDEV uint32_t search_codes8(const float2 (&x)[4], uint32_t t_addr) {
+  uint32_t acc = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float v = h ? x[j].y : x[j].x;
+      uint32_t c = v > lds_f32(t_addr + 7u * 4u) ? 8u : 0u;
+      c += v > lds_f32(t_addr + (c + 3u) * 4u) ? 4u : 0u;
+      c += v > lds_f32(t_addr + (c + 1u) * 4u) ? 2u : 0u;
+      c += v > lds_f32(t_addr + c * 4u) ? 1u : 0u;
+      acc |= c << (8 * j + 4 * h);
+    }
+  }
+  return acc;
+}
+
 // One CTA per 16384-weight group (256 blocks = one c1 scale), 256 threads;
 // 4 threads share a 64-weight block, 16 weights (32 bytes) each, 4 rounds.
+// kPoly: NF4's polynomial code search; otherwise the threshold search.
+template <bool kPoly>
 __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint16_t* __restrict__ W,
                                                                       int64_t n_blocks,
                                                                       uint2* __restrict__ codes,
@@ -136,8 +160,13 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
           x[k >> 2][k & 3] = make_float2(ratio_slow(__uint_as_float(w8[k] << 16), c),
                                          ratio_slow(__uint_as_float(w8[k] & 0xFFFF0000u), c));
       }
-      out[0] = nf4_codes8(x[0], P, t_addr);
-      out[1] = nf4_codes8(x[1], P, t_addr);
+      if (kPoly) {
+        out[0] = nf4_codes8(x[0], P, t_addr);
+        out[1] = nf4_codes8(x[1], P, t_addr);
+      } else {
+        out[0] = search_codes8(x[0], t_addr);
+        out[1] = search_codes8(x[1], t_addr);
+      }
       if ((u >> 2) < nblk) codes[blk0 * 4 + u] = make_uint2(out[0], out[1]);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (t & 31) == 0) report(status, QLORA_ERR_NONFINITE);
@@ -226,29 +255,34 @@ int num_sms() {
 }  // namespace
 
 cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
-                            int* status, cudaStream_t st) {
+                            int* status, int format, cudaStream_t st) {
   const int64_t n_blocks = n_weights / 64;
   const int64_t n_groups = (n_blocks + kGroupBlocks - 1) / kGroupBlocks;
   QuantParams qp;
-  const Nf4Tables& tab = nf4_tables();
-  if (!tab.poly_ok) return cudaErrorNotSupported;
+  const Nf4Tables& tab = code_tables(format);
+  const bool poly = format == 0;
+  if (poly && !tab.poly_ok) return cudaErrorNotSupported;
   for (int i = 0; i < 15; ++i) qp.t[i] = tab.t[i];
-  for (int k = 0; k < 6; ++k) qp.poly[k] = tab.poly[k];
+  for (int k = 0; k < 6; ++k) qp.poly[k] = poly ? tab.poly[k] : 0.0f;
   const int64_t grid = n_groups < (int64_t)num_sms() * 16 ? n_groups : (int64_t)num_sms() * 16;
-  nf4_quantize_kernel<<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint2*>(codes),
-                                                                 c2, c1, status, qp);
+  if (poly)
+    nf4_quantize_kernel<true><<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint2*>(codes),
+                                                                         c2, c1, status, qp);
+  else
+    nf4_quantize_kernel<false><<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint2*>(codes),
+                                                                          c2, c1, status, qp);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
-                           uint16_t* out, cudaStream_t st) {
+                           uint16_t* out, int format, cudaStream_t st) {
   const int64_t n_chunks = n_weights / 8;
   const int64_t want = (n_chunks + 256 * kDeqSteps - 1) / (256 * kDeqSteps);
   const int64_t cap = (int64_t)num_sms() * 8;
   const int64_t grid = want < cap ? (want > 0 ? want : 1) : cap;
   nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes), c2, c1, n_chunks,
-                                                     reinterpret_cast<uint4*>(out), nf4_tables());
+                                                     reinterpret_cast<uint4*>(out), code_tables(format));
   count_launches(1);
   return cudaGetLastError();
 }

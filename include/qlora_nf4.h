@@ -56,7 +56,25 @@ enum {
   QLORA_ERR_NONFINITE = -7,   /* device status: W holds an Inf or NaN */
   QLORA_ERR_TIMEOUT = -8,     /* device status: an internal wait expired */
   QLORA_ERR_DEVICE = -9,      /* current device is not sm_100 */
-  QLORA_ERR_SCRATCH_LIMIT = -10 /* problem needs more than the library's static scratch */
+  QLORA_ERR_SCRATCH_LIMIT = -10, /* problem needs more than the library's static scratch */
+  QLORA_ERR_FORMAT = -11        /* unknown code format, or reserved field not 0 */
+};
+
+/*
+ * 4-bit code formats.  NF4 is the method's own; FP4 and Int4 are the two
+ * formats the pages compare it with (nlp-lineage "QLoRA", section "What it
+ * showed", third bullet: "a standard 4-bit float" and "4-bit integers"),
+ * read as OCP E2M1 divided by 6 and as symmetric integers k/7.  All three
+ * use the same blocks, absmax scales and E4M3 double quantisation; a code is
+ * an index into the format's 16 ascending levels (qlora_code_levels), the
+ * nearest level to RN32(w / c_b), ties to the lower code.  FP4 and Int4 have
+ * 15 reachable levels; their lowest entry (-2 and -8/7) lies below -1 and is
+ * never produced.
+ */
+enum {
+  QLORA_FMT_NF4 = 0,
+  QLORA_FMT_FP4 = 1,
+  QLORA_FMT_INT4 = 2
 };
 
 /*
@@ -76,6 +94,8 @@ typedef struct qlora_nf4_weight {
   float* c1;
   int64_t n_rows; /* N: output features, >= 1 */
   int64_t n_cols; /* K: input features, a multiple of 64 */
+  int32_t format;   /* QLORA_FMT_*: the levels the codes index (0 = NF4) */
+  int32_t reserved; /* must be 0 */
 } qlora_nf4_weight;
 
 /* Bytes of codes, c2 and c1 for an N x K weight (sizes for the caller's
@@ -90,16 +110,22 @@ QLORA_API int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes,
  * (nlp-lineage "QLoRA", section "The idea", NF4 bullet). */
 QLORA_API int qlora_nf4_codebook(float levels[16]);
 
+/* The 16 levels of a code format (QLORA_FMT_*), ascending, as the kernels
+ * use them.  Returns QLORA_ERR_FORMAT for an unknown format. */
+QLORA_API int qlora_code_levels(int format, float levels[16]);
+
 /*
  * NF4 double quantisation of a bf16 weight W[N][K] (section "The idea",
  * NF4 and double-quantisation bullets).
  *   c_b   = max |w| over each block of 64 (fp32, exact)
  *   code  = nearest NF4 level to RN32(w / c_b), ties to the lower level
- *           (all-zero block: code 7, the exact zero)
+ *           (all-zero block: the code of the exact zero, 7 for NF4 and 8
+ *           for FP4 and Int4)
  *   c1_g  = RN32(max_{b in g} c_b / 448)      (groups of 256 blocks)
  *   c2_b  = E4M3_RNE_satfinite(RN32(c_b / c1_g)), 0 when c1_g = 0
  * W: device bf16[N*K].  out: descriptor whose buffers receive the result
- * (out->n_rows/n_cols are ignored and N, K used).  A non-finite weight sets
+ * (out->n_rows/n_cols are ignored and N, K used; out->format selects the
+ * levels, see QLORA_FMT_*).  A non-finite weight sets
  * *status_dev = QLORA_ERR_NONFINITE (the outputs are then unspecified).
  */
 QLORA_API int qlora_nf4_quantize(const uint16_t* W, int64_t N, int64_t K, const qlora_nf4_weight* out,

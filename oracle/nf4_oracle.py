@@ -26,6 +26,7 @@ import numpy as np
 __all__ = [
     "BLOCK", "DQ_BLOCK", "E4M3_MAX",
     "norm_cdf", "norm_ppf", "nf4_delta", "nf4_codebook_f64", "nf4_codebook",
+    "FORMATS", "fp4_codebook_f64", "int4_codebook_f64", "codebook",
     "nf4_midpoints", "nearest_level",
     "bf16_bits_to_f32", "f32_to_bf16_bits", "bf16_bits_to_f64",
     "e4m3_decode", "e4m3_encode", "e4m3_encode_exact",
@@ -105,6 +106,50 @@ def nf4_codebook_f64() -> list:
 def nf4_codebook() -> np.ndarray:
     """The codebook as stored and used: each fp64 level rounded to fp32."""
     return np.array(nf4_codebook_f64(), dtype=np.float32)
+
+
+# ---------------------------------------------------------------------------
+# The 4-bit formats NF4 is compared with (nlp-lineage "QLoRA", section "What it
+# showed", third bullet: "a standard 4-bit float" and "4-bit integers").  The
+# pages name them only; the readings below are the plainest ones.  Each keeps
+# everything else of the method (blocks of 64, absmax scale, E4M3 double
+# quantisation, nearest level with ties to the lower code) and swaps only the
+# 16 levels; a code is an index into the ascending level table.
+# ---------------------------------------------------------------------------
+
+FORMATS = ("nf4", "fp4", "int4")
+
+
+def fp4_codebook_f64() -> list:
+    """"A standard 4-bit float", read as OCP E2M1 (1 sign bit, 2 exponent bits
+    with bias 1, 1 mantissa bit: magnitudes 0, 1/2, 1, 3/2, 2, 3, 4, 6)
+    divided by its largest magnitude 6, so that the block absmax maps to +-1
+    as for NF4.  +0 and -0 are one level; the 16th entry is a pad level -2,
+    below every x = w / absmax (its decision midpoint -3/2 is never reached),
+    so the table stays 16 strictly increasing levels."""
+    mags = [Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3), Fraction(4), Fraction(6)]
+    pos = [m / 6 for m in mags]
+    return [-2.0] + [float(-p) for p in reversed(pos)] + [0.0] + [float(p) for p in pos]
+
+
+def int4_codebook_f64() -> list:
+    """"4-bit integers", read as symmetric absmax integer quantisation: levels
+    k/7 for k = -7 .. 7 (the block absmax maps to +-7), plus the code that
+    the symmetric form leaves unused (two's-complement -8) as the pad level
+    -8/7 (decision midpoint -15/14 < -1: never reached)."""
+    return [float(Fraction(k, 7)) for k in range(-8, 8)]
+
+
+def codebook(fmt: str = "nf4") -> np.ndarray:
+    """The 16 ascending fp32 levels of a format (each rounded once from its
+    exact or fp64 value)."""
+    if fmt == "nf4":
+        return nf4_codebook()
+    if fmt == "fp4":
+        return np.array(fp4_codebook_f64(), dtype=np.float32)
+    if fmt == "int4":
+        return np.array(int4_codebook_f64(), dtype=np.float32)
+    raise ValueError(f"unknown format {fmt!r}")
 
 
 def nf4_midpoints(q: np.ndarray | None = None) -> np.ndarray:
@@ -249,8 +294,9 @@ def _check_shape(N: int, K: int):
         raise ValueError("W must be [N, K] with K a multiple of 64")
 
 
-def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16):
-    """NF4 double quantisation of a bf16 weight ``[N, K]``.
+def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16, fmt: str = "nf4"):
+    """NF4 double quantisation of a bf16 weight ``[N, K]`` (``fmt`` swaps the
+    16 levels for one of the compared formats, see :func:`codebook`).
 
     Returns ``(codes, c2, c1)``:
       * ``codes`` uint8 ``[N*K/2]``: element 2j in the low nibble, 2j+1 in the
@@ -272,7 +318,7 @@ def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16):
     _check_shape(N, K)
     flat = W_bits.reshape(-1, BLOCK)
     nb = flat.shape[0]
-    q = nf4_codebook()
+    q = codebook(fmt)
     codes = np.empty((nb, BLOCK // 2), dtype=np.uint8)
     absmax = np.empty(nb, dtype=np.float32)
     for b0 in range(0, nb, chunk_blocks):
@@ -307,15 +353,16 @@ def decoded_scales(c2: np.ndarray, c1: np.ndarray) -> np.ndarray:
     return (dec * c1[g]).astype(np.float32)             # fp32 multiply
 
 
-def dequant(codes: np.ndarray, c2: np.ndarray, c1: np.ndarray, N: int, K: int) -> np.ndarray:
-    """doubleDequant(c1, c2, W_NF4) -> bf16 bits ``[N, K]``.
+def dequant(codes: np.ndarray, c2: np.ndarray, c1: np.ndarray, N: int, K: int, fmt: str = "nf4") -> np.ndarray:
+    """doubleDequant(c1, c2, W_NF4) -> bf16 bits ``[N, K]`` (``fmt``: the
+    levels the codes index, see :func:`codebook`).
 
     ("The idea", notation paragraph; inferensys: dequantised to BFloat16.)
     w^ = RNbf16(RN32(q_code * c^_b)) with c^_b from :func:`decoded_scales`:
     two fp32 multiplies, no fused multiply-add, then round to bf16.
     """
     _check_shape(N, K)
-    q = nf4_codebook()
+    q = codebook(fmt)
     cb = np.asarray(codes, dtype=np.uint8).reshape(-1, BLOCK // 2)
     code = np.empty((cb.shape[0], BLOCK), dtype=np.uint8)
     code[:, 0::2] = cb & 0xF

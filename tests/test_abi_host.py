@@ -93,3 +93,32 @@ def test_argument_checks_before_any_launch(q):
     assert L.qlora_nf4_quantize(fake, 64, 100, ctypes.byref(w), None, None) == -3
     assert L.qlora_nf4_quantize(None, 64, 128, ctypes.byref(w), None, None) == -1
     assert L.qlora_nf4_dequant(ctypes.byref(w_bad), fake, None, None) == -3
+
+
+def test_compared_format_levels_match_oracle_bitwise(q):
+    """FP4 (E2M1 / 6) and Int4 (k / 7) levels: the library's own host
+    derivation against the oracle's, bit for bit."""
+    for fmt in ("fp4", "int4"):
+        ours = np.array(q.codebook(fmt), dtype=np.float32)
+        ref = O.codebook(fmt)
+        assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32)), fmt
+    assert np.array_equal(np.array(q.codebook("nf4"), np.float32).view(np.uint32), O.nf4_codebook().view(np.uint32))
+
+
+def test_format_checks_before_any_launch(q):
+    """An unknown format or a nonzero reserved field is rejected on the host
+    (the fake pointers would fault if a kernel were launched)."""
+    L = q.lib()
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    arr = (ctypes.c_float * 16)()
+    assert L.qlora_code_levels(3, arr) == -11 and L.qlora_code_levels(-1, arr) == -11
+    for fmt, res in ((3, 0), (0, 1)):
+        w = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 128, fmt, res)
+        assert L.qlora_nf4_quantize(fake, 64, 128, ctypes.byref(w), None, None) == -11
+        assert L.qlora_nf4_dequant(ctypes.byref(w), fake, None, None) == -11
+        assert L.qlora_linear_fwd(fake, 4, ctypes.byref(w), fake, fake, 16, 1.0, fake, fake, fake, 1 << 20,
+                                  None, None) == -11
+        assert L.qlora_linear_bwd(fake, fake, 4, fake, ctypes.byref(w), fake, fake, 16, 1.0, fake, None, None,
+                                  fake, 1 << 20, None, None) == -11
+    assert "format" in q.status_string(-11)

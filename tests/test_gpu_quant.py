@@ -13,10 +13,10 @@ from bit_nf4_quantized_15_b200 import workloads as WL
 pytestmark = pytest.mark.gpu
 
 
-def gpu_quant(q, Wb):
+def gpu_quant(q, Wb, fmt="nf4"):
     W = from_bits(Wb)
     q.read_status()
-    w = q.quantize(W)
+    w = q.quantize(W, fmt=fmt)
     torch.cuda.synchronize()
     assert q.read_status() == 0
     return w
@@ -140,3 +140,41 @@ def test_roundtrip_2p31_sampled(lib):
         assert np.array_equal(bits(out.view(-1)[sl]), O.dequant(codes, c2, c1, 256, 64).reshape(-1))
     del W, out, w
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------- the compared formats (FP4, Int4)
+# nlp-lineage 'QLoRA', section 'What it showed', third bullet: NF4 against a
+# standard 4-bit float and 4-bit integers.  Same blocks and double
+# quantisation, other levels; the quantiser takes its threshold-search path.
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+@pytest.mark.parametrize("N,K,seed", [(1, 64, 10), (24, 192, 11), (37, 64 * 300, 12), (256, 4096, 13)])
+def test_formats_quantize_dequant_bitexact(lib, fmt, N, K, seed):
+    Wb = mixed_weights(N, K, seed)
+    ref = O.quantize(Wb, fmt=fmt)
+    w = gpu_quant(lib, Wb, fmt)
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, N, K, fmt=fmt))
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+def test_formats_every_significand_pair(lib, fmt):
+    Wb = mantissa_pair_matrix()
+    ref = O.quantize(Wb, fmt=fmt)
+    w = gpu_quant(lib, Wb, fmt)
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, *Wb.shape, fmt=fmt))
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+def test_formats_special_blocks(lib, fmt):
+    blocks = np.zeros((6, 64), np.float32)
+    blocks[1, 3] = 0.5
+    blocks[2, :] = -1.0
+    blocks[3, 0], blocks[3, 1], blocks[3, 2] = 1.0, 0.125, -0.125   # FP4 ties at 1/8
+    blocks[4, 0] = 3.0e38
+    blocks[5, :] = np.linspace(-1e-38, 1e-38, 64)
+    Wb = O.f32_to_bf16_bits(blocks)
+    ref = O.quantize(Wb, fmt=fmt)
+    w = gpu_quant(lib, Wb, fmt)
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, 6, 64, fmt=fmt))

@@ -1,0 +1,142 @@
+"""Pins for the oracle's two compared 4-bit formats (nlp-lineage "QLoRA",
+section "What it showed", third bullet: NF4 against "a standard 4-bit float"
+and "4-bit integers").
+
+The level tables are pinned against independent derivations: FP4 by decoding
+all 16 E2M1 bit patterns from the format's bit layout, Int4 by the exact
+rationals k/7, each rounded to fp32 by the exact-rational RN32 of
+``test_oracle_quant``.  The quantiser and dequantiser for each format are
+pinned against that file's brute-force rational implementations, given the
+pinned levels.
+"""
+
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle as O
+from test_oracle_quant import (_bf16, _halfgap, _tiny_inputs, bf16_value, brute_dequant, brute_quantize,
+                               rn32)
+
+
+def _e2m1_value(bits: int) -> Fraction:
+    """OCP E2M1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0;
+    exponent 0 is subnormal (m * 1/2)."""
+    s, e, m = (bits >> 3) & 1, (bits >> 1) & 3, bits & 1
+    mag = Fraction(m, 2) if e == 0 else (1 + Fraction(m, 2)) * Fraction(2) ** (e - 1)
+    return -mag if s else mag
+
+
+def _as_f32(fr: Fraction) -> np.float32:
+    v = np.float32(float(fr))
+    assert Fraction(float(v)) == fr, "value must be representable"
+    return v
+
+
+def test_fp4_levels_are_e2m1_over_6():
+    vals = sorted({_e2m1_value(b) for b in range(16)})          # +0 and -0 collapse: 15 values
+    assert len(vals) == 15 and max(vals) == 6 and min(vals) == -6
+    want = [_as_f32(rn32(v / 6)) for v in vals]
+    q = O.codebook("fp4")
+    assert q.dtype == np.float32 and q.shape == (16,)
+    assert np.array_equal(q[1:].view(np.uint32), np.array(want, np.float32).view(np.uint32))
+    assert q[0] < -1 and (float(q[0]) + float(q[1])) / 2 < -1  # pad level never chosen
+    assert q[8] == 0 and q[15] == 1 and q[1] == -1
+
+
+def test_int4_levels_are_k_over_7():
+    want = [_as_f32(rn32(Fraction(k, 7))) for k in range(-7, 8)]
+    q = O.codebook("int4")
+    assert np.array_equal(q[1:].view(np.uint32), np.array(want, np.float32).view(np.uint32))
+    assert (float(q[0]) + float(q[1])) / 2 < -1
+    gaps = np.diff(q[1:].astype(np.float64))
+    assert np.all(np.abs(gaps - 1 / 7) < 2 ** -23)              # uniform spacing up to fp32 rounding
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+def test_levels_strictly_increasing_with_zero(fmt):
+    q = O.codebook(fmt).astype(np.float64)
+    assert np.all(np.diff(q) > 0) and 0.0 in q and q[-1] == 1.0
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+@pytest.mark.parametrize("case", range(3))
+def test_quantize_matches_bruteforce(fmt, case):
+    W = _tiny_inputs()[case]
+    a = O.quantize(W, fmt=fmt)
+    b = brute_quantize(W, O.codebook(fmt))
+    for x, y in zip(a, b):
+        assert np.array_equal(np.asarray(x).view(np.uint8), np.asarray(y).view(np.uint8))
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+@pytest.mark.parametrize("case", range(3))
+def test_dequant_matches_bruteforce(fmt, case):
+    W = _tiny_inputs()[case]
+    N, K = W.shape
+    codes, c2, c1 = O.quantize(W, fmt=fmt)
+    assert np.array_equal(O.dequant(codes, c2, c1, N, K, fmt=fmt),
+                          brute_dequant(codes, c2, c1, N, K, O.codebook(fmt)))
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+def test_special_blocks(fmt):
+    blk = np.zeros(64, np.float32)
+    blk[0], blk[1], blk[2] = 0.5, -0.5, 0.0
+    codes, c2, c1 = O.quantize(_bf16(blk).reshape(1, 64), fmt=fmt)
+    assert codes[0] & 15 == 15 and codes[0] >> 4 == 1 and codes[1] & 15 == 8   # +c, -c, 0
+    codes, c2, c1 = O.quantize(np.zeros((2, 64), np.uint16), fmt=fmt)
+    assert np.all(codes == 0x88) and np.all(O.dequant(codes, c2, c1, 2, 64, fmt=fmt) == 0)
+
+
+def test_fp4_ties_go_to_lower_level():
+    """x = 1/8 lies exactly between the FP4 levels 1/12 and 1/6 (in fp32:
+    both levels and the midpoint are checked exactly) -> the lower one."""
+    q = O.codebook("fp4").astype(np.float64)
+    mid = (q[9] + q[10]) / 2
+    if float(np.float32(mid)) == mid:
+        assert O.nearest_level(np.array([np.float32(mid)]), O.codebook("fp4"))[0] == 9
+    x = np.float32(0.125)   # w / c = 1/8 exactly
+    code = O.nearest_level(np.array([x]), O.codebook("fp4"))[0]
+    d9, d10 = abs(Fraction(float(x)) - Fraction(q[9])), abs(Fraction(float(x)) - Fraction(q[10]))
+    assert code == (9 if d9 <= d10 else 10)
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+def test_round_trip_error_bound(fmt):
+    rng = np.random.default_rng(15)
+    n = 64 * 1024
+    a = rng.normal(0, 0.02, n // 2)
+    t = rng.standard_t(3, n // 2) * 0.02
+    t *= np.where(rng.random(n // 2) < 0.001, 50.0, 1.0)
+    W = _bf16(np.concatenate([a, t])).reshape(64, -1)
+    N, K = W.shape
+    codes, c2, c1 = O.quantize(W, fmt=fmt)
+    What = O.bf16_bits_to_f64(O.dequant(codes, c2, c1, N, K, fmt=fmt)).reshape(-1)
+    w = O.bf16_bits_to_f64(W).reshape(-1)
+    q = O.codebook(fmt)
+    code = np.empty(n, np.uint8)
+    code[0::2], code[1::2] = codes & 15, codes >> 4
+    assert np.all(code >= 1)                                   # the pad level is never used
+    c = np.repeat(O.block_absmax(W).astype(np.float64), 64)
+    chat = np.repeat(O.decoded_scales(c2, c1).astype(np.float64), 64)
+    hg = np.array([_halfgap(q, k) for k in range(16)])[code]
+    qv = q.astype(np.float64)[code]
+    bound = (c * (hg + 2.0 ** -24) + np.abs(qv) * np.abs(chat - c)
+             + np.abs(qv * chat) * 2.0 ** -24 + np.abs(What) * 2.0 ** -8 + 1e-45)
+    assert np.all(np.abs(w - What) <= bound * (1 + 1e-12))
+
+
+def test_nf4_beats_the_compared_formats_on_normal_weights():
+    """The pages' ranking (NF4 ahead of FP4 and Int4) holds for the
+    quantisation error these readings give on normally distributed weights."""
+    rng = np.random.default_rng(16)
+    W = _bf16(rng.normal(0, 0.02, (64, 64 * 64)))
+    N, K = W.shape
+    w = O.bf16_bits_to_f64(W)
+    err = {}
+    for f in O.FORMATS:
+        What = O.bf16_bits_to_f64(O.dequant(*O.quantize(W, fmt=f), N, K, fmt=f))
+        err[f] = float(np.mean((w - What) ** 2))
+    assert err["nf4"] < err["fp4"] and err["nf4"] < err["int4"]

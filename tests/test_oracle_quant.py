@@ -69,8 +69,8 @@ def bf16_value(bits: int) -> Fraction:
     return Fraction(float(O.bf16_bits_to_f32(np.array([bits], np.uint16))[0]))
 
 
-def brute_quantize(W_bits: np.ndarray):
-    q = [Fraction(float(v)) for v in O.nf4_codebook()]
+def brute_quantize(W_bits: np.ndarray, levels=None):
+    q = [Fraction(float(v)) for v in (O.nf4_codebook() if levels is None else levels)]
     mids = [(q[i] + q[i + 1]) / 2 for i in range(15)]
     flat = W_bits.reshape(-1).tolist()
     nb = len(flat) // 64
@@ -97,8 +97,8 @@ def brute_quantize(W_bits: np.ndarray):
             np.array([float(v) for v in c1], np.float32))
 
 
-def brute_dequant(codes, c2, c1, N, K):
-    q = [Fraction(float(v)) for v in O.nf4_codebook()]
+def brute_dequant(codes, c2, c1, N, K, levels=None):
+    q = [Fraction(float(v)) for v in (O.nf4_codebook() if levels is None else levels)]
     out = np.empty(N * K, np.uint16)
     for idx in range(N * K):
         code = (int(codes[idx // 2]) >> (4 * (idx & 1))) & 15
