@@ -371,9 +371,9 @@ def run_ours(args):
     qb, db = quant_bytes(rt_N, rt_K), dequant_bytes(rt_N, rt_K)
     reps = max(args.steps, 3)
 
-    def roundtrip(fmt):
+    def roundtrip(fmt, scale="e4m3"):
         """(quantise GB/s, dequantise GB/s) of one format on the round trip."""
-        wrt = q.NF4Weight.empty(rt_N, rt_K, dev, fmt)
+        wrt = q.NF4Weight.empty(rt_N, rt_K, dev, fmt, scale)
         for _ in range(2):
             q.quantize_into(Wrt, wrt)
             q.dequant(wrt, out=Wout)
@@ -395,10 +395,10 @@ def run_ours(args):
     quant_gbs, dequant_gbs = roundtrip("nf4")
     # the two 4-bit formats the method is compared with (same round trip)
     formats = {}
-    for fmt in ("fp4", "int4"):
-        qg, dg = roundtrip(fmt)
-        formats[fmt] = {"quant_gbs": qg, "quant_frac": qg / pk["hbm_gbs"], "dequant_gbs": dg,
-                        "dequant_frac": dg / pk["hbm_gbs"]}
+    for fmt, scale in (("fp4", "e4m3"), ("int4", "e4m3"), ("nf4", "e5m2")):
+        qg, dg = roundtrip(fmt, scale)
+        formats[fmt if scale == "e4m3" else f"{fmt}_{scale}"] = {
+            "quant_gbs": qg, "quant_frac": qg / pk["hbm_gbs"], "dequant_gbs": dg, "dequant_frac": dg / pk["hbm_gbs"]}
     del Wrt, Wout
     assert q.read_status(dev) == 0
 
@@ -456,7 +456,8 @@ def run_ours(args):
                       "bytes": qb, "peak_source": f"{pk_kind} HBM copy"},
             "dequant": {"workload": RT_WORKLOAD, "value": dequant_gbs, "unit": "GB/s", "frac": dequant_gbs / hbm, "peak": hbm,
                         "bytes": db, "peak_source": f"{pk_kind} HBM copy"},
-            "formats": {"workload": RT_WORKLOAD + "; FP4 = E2M1/6 and Int4 = k/7 levels (the compared formats)",
+            "formats": {"workload": RT_WORKLOAD + "; FP4 = E2M1/6 and Int4 = k/7 levels (the compared formats), "
+                                                  "nf4_e5m2 = NF4 with E5M2 block scales",
                         "unit": "GB/s", **formats},
             "gemv": gemv,
             "cpu_baseline": base,

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "lib", "NF4Weight", "quantize", "quantize_into", "dequant", "workspace_bytes", "linear_fwd", "linear_bwd",
-    "codebook", "FORMATS", "status_string", "kernel_launches", "set_gemm_events", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
+    "codebook", "FORMATS", "SCALES", "status_string", "kernel_launches", "set_gemm_events", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
@@ -34,6 +34,9 @@ QLORA_ERR_TIMEOUT = -8
 # Code formats (QLORA_FMT_*): NF4, and the two 4-bit formats the method is
 # compared with (FP4 = E2M1/6, Int4 = k/7).
 FORMATS = {"nf4": 0, "fp4": 1, "int4": 2}
+# Codec of the 8-bit block scales c2 (QLORA_SCALE_*): E4M3, or E5M2 as the
+# compared alternative.
+SCALES = {"e4m3": 0, "e5m2": 1}
 
 
 class QLoRAError(RuntimeError):
@@ -43,7 +46,7 @@ class QLoRAError(RuntimeError):
 class qlora_nf4_weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p),
                 ("n_rows", ctypes.c_int64), ("n_cols", ctypes.c_int64),
-                ("format", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("format", ctypes.c_int32), ("scale_codec", ctypes.c_int32)]
 
 
 _lib = None
@@ -154,30 +157,32 @@ def storage_bytes(N: int, K: int):
 @dataclass
 class NF4Weight:
     """Quantized weight: codes uint8[N*K/2], c2 uint8[N*K/64] (E4M3), c1 float32[ceil(N*K/16384)];
-    ``fmt`` names the 16 levels the codes index (see FORMATS)."""
+    ``fmt`` names the 16 levels the codes index (see FORMATS), ``scale`` the
+    8-bit float of c2 (see SCALES)."""
     codes: torch.Tensor
     c2: torch.Tensor
     c1: torch.Tensor
     N: int
     K: int
     fmt: str = "nf4"
+    scale: str = "e4m3"
 
     def descriptor(self) -> qlora_nf4_weight:
-        if self.fmt not in FORMATS:
-            raise QLoRAError(f"unknown format {self.fmt!r}")
+        if self.fmt not in FORMATS or self.scale not in SCALES:
+            raise QLoRAError(f"unknown format {self.fmt!r} or scale codec {self.scale!r}")
         return qlora_nf4_weight(self.codes.data_ptr(), self.c2.data_ptr(), self.c1.data_ptr(), self.N, self.K,
-                                FORMATS[self.fmt], 0)
+                                FORMATS[self.fmt], SCALES[self.scale])
 
     @property
     def device(self):
         return self.codes.device
 
     @staticmethod
-    def empty(N: int, K: int, device="cuda", fmt: str = "nf4") -> "NF4Weight":
+    def empty(N: int, K: int, device="cuda", fmt: str = "nf4", scale: str = "e4m3") -> "NF4Weight":
         nc, n2, n1 = storage_bytes(N, K)
         return NF4Weight(torch.empty(nc, dtype=torch.uint8, device=device),
                          torch.empty(n2, dtype=torch.uint8, device=device),
-                         torch.empty(n1 // 4, dtype=torch.float32, device=device), N, K, fmt)
+                         torch.empty(n1 // 4, dtype=torch.float32, device=device), N, K, fmt, scale)
 
 
 def codebook(fmt: str = "nf4"):
@@ -198,12 +203,13 @@ def quantize_into(W: torch.Tensor, out: NF4Weight, status=None):
     return out
 
 
-def quantize(W: torch.Tensor, status=None, fmt: str = "nf4") -> NF4Weight:
+def quantize(W: torch.Tensor, status=None, fmt: str = "nf4", scale: str = "e4m3") -> NF4Weight:
     """NF4 double quantisation of a bf16 CUDA weight [N, K] (K % 64 == 0);
-    fmt="fp4" or "int4" quantises to one of the compared formats instead."""
+    fmt="fp4" or "int4" quantises to one of the compared formats instead,
+    scale="e5m2" stores the block scales as E5M2."""
     _bf16_cuda(W, "W")
     N, K = W.shape
-    return quantize_into(W, NF4Weight.empty(N, K, W.device, fmt), status)
+    return quantize_into(W, NF4Weight.empty(N, K, W.device, fmt, scale), status)
 
 
 def dequant(w: NF4Weight, out: torch.Tensor | None = None, status=None) -> torch.Tensor:

@@ -99,11 +99,14 @@ EpiArgs epi_none() {
   return e;
 }
 
-bool format_ok(const qlora_nf4_weight* w) { return w->format >= 0 && w->format < kNumFormats && w->reserved == 0; }
+bool format_ok(const qlora_nf4_weight* w) {
+  return w->format >= 0 && w->format < kNumFormats && (w->scale_codec == QLORA_SCALE_E4M3 || w->scale_codec == QLORA_SCALE_E5M2);
+}
 
-void fill_common(EngineArgs* a, int* status, int format) {
+void fill_common(EngineArgs* a, int* status, int format, int scale_codec) {
   std::memset(a, 0, sizeof(*a));
   a->status = status;
+  a->c2_e5m2 = scale_codec == QLORA_SCALE_E5M2;
   const Nf4Tables& t = code_tables(format);
   for (int i = 0; i < 16; ++i) a->q[i] = t.q[i];
 }
@@ -203,7 +206,7 @@ const char* qlora_status_string(int code) {
     case QLORA_ERR_NONFINITE: return "weight holds an Inf or NaN";
     case QLORA_ERR_TIMEOUT: return "an internal GPU wait expired";
     case QLORA_ERR_DEVICE: return "current device is not an sm_100 GPU";
-    case QLORA_ERR_FORMAT: return "unknown code format (QLORA_FMT_*) or nonzero reserved field";
+    case QLORA_ERR_FORMAT: return "unknown code format (QLORA_FMT_*) or scale codec (QLORA_SCALE_*)";
     case QLORA_ERR_SCRATCH_LIMIT: return "problem needs more workspace than the library's 8 MiB static scratch";
   }
   return "unknown status";
@@ -250,7 +253,8 @@ int qlora_nf4_quantize(const uint16_t* W, int64_t N, int64_t K, const qlora_nf4_
   DevInfo di;
   if (int rc = current_device_info(&di)) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return launch_quantize(W, N * K, out->codes, out->c2, out->c1, status_dev, out->format, st) == cudaSuccess
+  return launch_quantize(W, N * K, out->codes, out->c2, out->c1, status_dev, out->format, out->scale_codec, st) ==
+                 cudaSuccess
              ? QLORA_OK
              : QLORA_ERR_CUDA;
 }
@@ -264,7 +268,8 @@ int qlora_nf4_dequant(const qlora_nf4_weight* w, uint16_t* W_out, int* status_de
   DevInfo di;
   if (int rc = current_device_info(&di)) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return launch_dequant(w->codes, w->c2, w->c1, w->n_rows * w->n_cols, W_out, w->format, st) == cudaSuccess
+  return launch_dequant(w->codes, w->c2, w->c1, w->n_rows * w->n_cols, W_out, w->format, w->scale_codec, st) ==
+                 cudaSuccess
              ? QLORA_OK
              : QLORA_ERR_CUDA;
 }
@@ -324,6 +329,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
     ga.T_save = T_save;
     ga.status = status_dev;
     const Nf4Tables& tb = code_tables(w->format);
+    ga.c2_e5m2 = w->scale_codec == QLORA_SCALE_E5M2;
     for (int i = 0; i < 16; ++i) ga.q[i] = tb.q[i];
     cudaEvent_t e0 = g_ev_start, e1 = g_ev_end;
     g_ev_start = g_ev_end = nullptr;
@@ -336,7 +342,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
   // (1) T = X.L1 (fp32, saved) and s.T in bf16 for the LoRA extension.
   {
     EngineArgs a;
-    fill_common(&a, status_dev, w->format);
+    fill_common(&a, status_dev, w->format, w->scale_codec);
     const GemmPlan& p = lay.t_fwd;
     if (map_operand(&a.tmA, X, 0, M, K, 128) || map_operand(&a.tmB, L1, 1, r, K, p.BN)) return QLORA_ERR_CUDA;
     a.rows = (int)M;
@@ -356,7 +362,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
   // (2) Y^T = W^.X^T + L2^T.(s.T)^T, W^ dequantised on chip.
   {
     EngineArgs a;
-    fill_common(&a, status_dev, w->format);
+    fill_common(&a, status_dev, w->format, w->scale_codec);
     const GemmPlan& p = lay.y_fwd;
     const int kb_ext = (r + 63) / 64;
     const bool pair = use_pair_fwd(p, (int)N, (int)M, kb_ext);
@@ -412,7 +418,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const flo
   // (1) dT = dY.L2^T, kept as s.dT in bf16.
   {
     EngineArgs a;
-    fill_common(&a, status_dev, w->format);
+    fill_common(&a, status_dev, w->format, w->scale_codec);
     const GemmPlan& p = lay.dt;
     if (map_operand(&a.tmA, dY, 0, M, N, 128) || map_operand(&a.tmB, L2, 0, r, N, p.BN)) return QLORA_ERR_CUDA;
     a.rows = (int)M;
@@ -428,7 +434,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const flo
   // (2) dX^T = W^T.dY^T + L1.(s.dT)^T, W^ dequantised on chip (MN-major).
   if (dX) {
     EngineArgs a;
-    fill_common(&a, status_dev, w->format);
+    fill_common(&a, status_dev, w->format, w->scale_codec);
     const GemmPlan& p = lay.dx;
     if (map_codes(&a.tmA, w->codes, N, K, 1) || map_operand(&a.tmB, dY, 0, M, N, p.BN) ||
         map_operand(&a.tmAx, L1, 0, K, r, 128) || map_operand(&a.tmBx, sdT, 0, M, r, p.BN))
@@ -451,7 +457,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const flo
   // (3) dL1 = X^T.(s.dT): rows k, reduction over tokens.
   if (dL1) {
     EngineArgs a;
-    fill_common(&a, status_dev, w->format);
+    fill_common(&a, status_dev, w->format, w->scale_codec);
     const GemmPlan& p = lay.dl1;
     if (map_operand(&a.tmA, X, 1, K, M, 128) || map_operand(&a.tmB, sdT, 1, r, M, p.BN)) return QLORA_ERR_CUDA;
     a.rows = (int)K;
@@ -468,7 +474,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const flo
   // (4) dL2^T = dY^T.(s.T): rows n, reduction over tokens, stored as dL2[r][N].
   if (dL2) {
     EngineArgs a;
-    fill_common(&a, status_dev, w->format);
+    fill_common(&a, status_dev, w->format, w->scale_codec);
     const GemmPlan& p = lay.dl2;
     if (map_operand(&a.tmA, dY, 1, N, M, 128) || map_operand(&a.tmB, sT, 1, r, M, p.BN)) return QLORA_ERR_CUDA;
     a.rows = (int)N;

@@ -201,8 +201,15 @@ QDEV float e4m3_to_float(uint32_t code) {
   return __half2float(__half(hr));
 }
 
-// Decoded block scale c^ = RN32(dec(c2) * c1).
-QDEV float decode_scale(uint32_t c2code, float c1v) { return __fmul_rn(e4m3_to_float(c2code), c1v); }
+// E5M2 code -> fp32 (exact: an E5M2 byte is the high byte of the fp16 of the
+// same value).
+QDEV float e5m2_to_float(uint32_t code) { return __half2float(__ushort_as_half((unsigned short)(code << 8))); }
+
+// Decoded block scale c^ = RN32(dec(c2) * c1); c2 is E4M3, or E5M2 for the
+// scale-codec variant.
+QDEV float decode_scale(uint32_t c2code, float c1v, bool e5m2 = false) {
+  return __fmul_rn(e5m2 ? e5m2_to_float(c2code) : e4m3_to_float(c2code), c1v);
+}
 
 QDEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const uint32_t taddr = tlane + (uint32_t)(s * 32);
         const uint8_t* ctile = smem + s * L::STAGE + kA + L::B + rl * 32;
-        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        const float chat = valid ? decode_scale(c2raw, c1v, args.c2_e5m2 != 0) : 0.0f;
         if (valid && it + R::G < my_kb) {  // this group's next scale, one round ahead
           const int64_t f = n * bpr + kb_lo + it + R::G;
           c2raw = __ldg(args.c2 + f);
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const int64_t nn = (int64_t)(kb_lo + it) * 64 + nl;
         const bool valid = kvalid && nn < args.wN;
-        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        const float chat = valid ? decode_scale(c2raw, c1v, args.c2_e5m2 != 0) : 0.0f;
         if (it + kStages < my_kb) {
           const int64_t nx = nn + 64 * kStages;
           c2raw = 0;

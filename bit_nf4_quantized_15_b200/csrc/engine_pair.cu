@@ -312,7 +312,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         const uint32_t ph = (uint32_t)(it / kPA) & 1u;
         const uint32_t taddr = tlane + (uint32_t)(a * 32);
         const uint4 c0 = cn0, c1 = cn1;
-        const float chat = valid ? decode_scale(c2raw, c1v) : 0.0f;
+        const float chat = valid ? decode_scale(c2raw, c1v, args.c2_e5m2 != 0) : 0.0f;
         if (valid && it + kPG < n_kb) {  // this group's next codes and scale, one round ahead
           const int64_t f = n * bpr + it + kPG;
           cn0 = __ldg(crow + 2 * (it + kPG));

@@ -177,9 +177,9 @@ QDEV RowScales load_row_scales(const GemvArgs& a, int rt, int un, int rl) {
   return s;
 }
 // c^ of k block q (0..3) of the unit whose first block is f0's.
-QDEV float row_chat(const RowScales& s, int q, int64_t f0) {
+QDEV float row_chat(const RowScales& s, int q, int64_t f0, bool e5m2) {
   const float c1 = ((f0 + q) >> 8) == (f0 >> 8) ? s.c1a : s.c1b;
-  return decode_scale((s.c2 >> (8 * q)) & 0xFFu, c1);
+  return decode_scale((s.c2 >> (8 * q)) & 0xFFu, c1, e5m2);
 }
 
 // NT = 8-token column tiles (1 for M <= 8, 2 for M <= 16).
@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
               cw[e] = lds64(st + (uint32_t)rl * 128 +
                             ((((uint32_t)(2 * q + (cq >> 1))) ^ (uint32_t)(rl & 7)) << 4) + 8u * (uint32_t)(cq & 1));
               const int64_t f0 = ((int64_t)rt * 128 + rl) * args.kbt + (int64_t)un * kUnitKB;
-              const float ch = row_chat(cur[2 * h + e], q, f0);
+              const float ch = row_chat(cur[2 * h + e], q, f0, args.c2_e5m2 != 0);
               cc[e] = make_float2(ch, ch);
             }
 #pragma unroll

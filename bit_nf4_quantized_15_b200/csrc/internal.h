@@ -66,6 +66,7 @@ struct EngineArgs {
   CUtensorMap tmBx;  // extension B
   const uint8_t* codes;  // NF4 codes [wN][wK/2] (read directly by the pair forward)
   const uint8_t* c2;
+  int c2_e5m2;           // c2 holds E5M2 codes instead of E4M3
   const float* c1;
   int64_t wN, wK;    // quantised weight shape (for scale indexing)
   int rows, cols;    // output extent: UMMA-M side, UMMA-N side
@@ -129,6 +130,7 @@ struct GemvArgs {
   CUtensorMap tmCodes;  // uint8 [N][K/2], box 128 x 128, 128-byte swizzle
   CUtensorMap tmX;      // bf16 [M][K], box 64 x 16, 128-byte swizzle
   const uint8_t* c2;
+  int c2_e5m2;          // c2 holds E5M2 codes instead of E4M3
   const float* c1;
   int64_t N, K;
   int M;
@@ -152,9 +154,9 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& p, const uint16_t* X,
 
 // --------------------------------------------------------- quantise kernels
 cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
-                            int* status, int format, cudaStream_t st);
+                            int* status, int format, int scale_codec, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
-                           uint16_t* out, int format, cudaStream_t st);
+                           uint16_t* out, int format, int scale_codec, cudaStream_t st);
 cudaError_t launch_scale_to_bf16(const float* in, int64_t n, float s, uint16_t* out, cudaStream_t st);
 
 }  // namespace qnf4

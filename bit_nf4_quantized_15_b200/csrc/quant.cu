@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
                                                                       uint2* __restrict__ codes,
                                                                       uint8_t* __restrict__ c2,
                                                                       float* __restrict__ c1, int* status,
-                                                                      QuantParams qp) {
+                                                                      QuantParams qp, int e5m2) {
   __shared__ float s_t[16];
   __shared__ float s_absmax[kGroupBlocks];
   __shared__ float s_wmax[kQuantThreads / 32];
@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (t & 31) == 0) report(status, QLORA_ERR_NONFINITE);
     __syncthreads();
-    // second level: c1 = RN32(max c_b / 448), c2_b = E4M3(RN32(c_b / c1))
+    // second level: c1 = RN32(max c_b / 448), c2_b = E4M3(RN32(c_b / c1));
+    // for E5M2 scale codes 57344 and E5M2
     float cb = t < nblk ? s_absmax[t] : 0.0f;
     float wm = cb;
 #pragma unroll
@@ -181,11 +182,12 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
     float gmax = s_wmax[0];
 #pragma unroll
     for (int k = 1; k < kQuantThreads / 32; ++k) gmax = fmaxf(gmax, s_wmax[k]);
-    const float c1v = __fdiv_rn(gmax, 448.0f);
+    const float c1v = __fdiv_rn(gmax, e5m2 ? 57344.0f : 448.0f);
     if (t == 0) c1[g] = c1v;
     if (t < nblk) {
       uint8_t code = 0;
-      if (c1v > 0.0f) code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(cb, c1v), __NV_SATFINITE, __NV_E4M3);
+      if (c1v > 0.0f)
+        code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(cb, c1v), __NV_SATFINITE, e5m2 ? __NV_E5M2 : __NV_E4M3);
       c2[blk0 + t] = code;
     }
     __syncthreads();
@@ -201,7 +203,7 @@ constexpr int kDeqSteps = 8;
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ codes,
                                                           const uint8_t* __restrict__ c2,
                                                           const float* __restrict__ c1, int64_t n_chunks,
-                                                          uint4* __restrict__ out, Nf4Tables tab) {
+                                                          uint4* __restrict__ out, Nf4Tables tab, int e5m2) {
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = tab.q[threadIdx.x];
   __syncthreads();
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __rest
     for (int u = 0; u < kDeqSteps; ++u) {
       const int64_t ci = c0 + u * stride;
       if (ci < n_chunks) {
-        const float chat = decode_scale(s2[u], s1[u]);
+        const float chat = decode_scale(s2[u], s1[u], e5m2 != 0);
         const float2 cc = make_float2(chat, chat);
         uint32_t o[4];
 #pragma unroll
@@ -255,7 +257,7 @@ int num_sms() {
 }  // namespace
 
 cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
-                            int* status, int format, cudaStream_t st) {
+                            int* status, int format, int scale_codec, cudaStream_t st) {
   const int64_t n_blocks = n_weights / 64;
   const int64_t n_groups = (n_blocks + kGroupBlocks - 1) / kGroupBlocks;
   QuantParams qp;
@@ -267,22 +269,22 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes
   const int64_t grid = n_groups < (int64_t)num_sms() * 16 ? n_groups : (int64_t)num_sms() * 16;
   if (poly)
     nf4_quantize_kernel<true><<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint2*>(codes),
-                                                                         c2, c1, status, qp);
+                                                                         c2, c1, status, qp, scale_codec);
   else
     nf4_quantize_kernel<false><<<(unsigned)grid, kQuantThreads, 0, st>>>(W, n_blocks, reinterpret_cast<uint2*>(codes),
-                                                                          c2, c1, status, qp);
+                                                                          c2, c1, status, qp, scale_codec);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float* c1, int64_t n_weights,
-                           uint16_t* out, int format, cudaStream_t st) {
+                           uint16_t* out, int format, int scale_codec, cudaStream_t st) {
   const int64_t n_chunks = n_weights / 8;
   const int64_t want = (n_chunks + 256 * kDeqSteps - 1) / (256 * kDeqSteps);
   const int64_t cap = (int64_t)num_sms() * 8;
   const int64_t grid = want < cap ? (want > 0 ? want : 1) : cap;
   nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes), c2, c1, n_chunks,
-                                                     reinterpret_cast<uint4*>(out), code_tables(format));
+                                                     reinterpret_cast<uint4*>(out), code_tables(format), scale_codec);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -57,7 +57,7 @@ enum {
   QLORA_ERR_TIMEOUT = -8,     /* device status: an internal wait expired */
   QLORA_ERR_DEVICE = -9,      /* current device is not sm_100 */
   QLORA_ERR_SCRATCH_LIMIT = -10, /* problem needs more than the library's static scratch */
-  QLORA_ERR_FORMAT = -11        /* unknown code format, or reserved field not 0 */
+  QLORA_ERR_FORMAT = -11        /* unknown code format or scale codec */
 };
 
 /*
@@ -78,6 +78,19 @@ enum {
 };
 
 /*
+ * Codec of the 8-bit block scales c2.  The pages say only that the scales
+ * become 8-bit floats; E4M3 (max 448) is the reading taken, E5M2 (max 57344:
+ * two more exponent bits, one fewer mantissa bit) the compared alternative.
+ * With E5M2, c1_g = RN32(max c_b / 57344) and c2_b = E5M2_RNE_satfinite(
+ * RN32(c_b / c1_g)); the dequantiser decodes accordingly.  Codes and storage
+ * are unchanged.
+ */
+enum {
+  QLORA_SCALE_E4M3 = 0,
+  QLORA_SCALE_E5M2 = 1
+};
+
+/*
  * The quantized weight (nlp-lineage "QLoRA", section "The idea": blocks of
  * 64 weights, 4-bit NormalFloat codes, 8-bit block scales c2 and 32-bit
  * second-level scales c1; inferensys glossary "QLoRA": the scales become
@@ -94,8 +107,8 @@ typedef struct qlora_nf4_weight {
   float* c1;
   int64_t n_rows; /* N: output features, >= 1 */
   int64_t n_cols; /* K: input features, a multiple of 64 */
-  int32_t format;   /* QLORA_FMT_*: the levels the codes index (0 = NF4) */
-  int32_t reserved; /* must be 0 */
+  int32_t format;      /* QLORA_FMT_*: the levels the codes index (0 = NF4) */
+  int32_t scale_codec; /* QLORA_SCALE_*: the 8-bit float of c2 (0 = E4M3) */
 } qlora_nf4_weight;
 
 /* Bytes of codes, c2 and c1 for an N x K weight (sizes for the caller's
@@ -125,7 +138,7 @@ QLORA_API int qlora_code_levels(int format, float levels[16]);
  *   c2_b  = E4M3_RNE_satfinite(RN32(c_b / c1_g)), 0 when c1_g = 0
  * W: device bf16[N*K].  out: descriptor whose buffers receive the result
  * (out->n_rows/n_cols are ignored and N, K used; out->format selects the
- * levels, see QLORA_FMT_*).  A non-finite weight sets
+ * levels, see QLORA_FMT_*, and out->scale_codec the c2 codec, QLORA_SCALE_*).  A non-finite weight sets
  * *status_dev = QLORA_ERR_NONFINITE (the outputs are then unspecified).
  */
 QLORA_API int qlora_nf4_quantize(const uint16_t* W, int64_t N, int64_t K, const qlora_nf4_weight* out,

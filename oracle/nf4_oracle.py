@@ -30,6 +30,7 @@ __all__ = [
     "nf4_midpoints", "nearest_level",
     "bf16_bits_to_f32", "f32_to_bf16_bits", "bf16_bits_to_f64",
     "e4m3_decode", "e4m3_encode", "e4m3_encode_exact",
+    "E5M2_MAX", "SCALE_CODECS", "e5m2_decode", "e5m2_encode", "e5m2_encode_exact",
     "block_absmax", "quantize", "dequant", "decoded_scales",
     "linear_fwd", "linear_bwd", "adapter_grads",
     "storage_bytes", "bits_per_weight",
@@ -38,6 +39,7 @@ __all__ = [
 BLOCK = 64          # weights per first-level block ("The idea": blocks of 64)
 DQ_BLOCK = 256      # first-level scales per second-level (c1) block
 E4M3_MAX = 448.0    # largest finite OCP E4M3 value
+E5M2_MAX = 57344.0  # largest finite OCP E5M2 value
 
 
 # ---------------------------------------------------------------------------
@@ -279,6 +281,91 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# E5M2: the other 8-bit float, for the scale-codec variant of the double
+# quantisation (the pages say only "8-bit floats"; E4M3 is the method's
+# reading here, E5M2 the compared alternative: two more exponent bits, one
+# fewer mantissa bit).
+# ---------------------------------------------------------------------------
+
+def e5m2_decode(code: np.ndarray) -> np.ndarray:
+    """OCP FP8 E5M2 (bias 15; exponent 31 holds Inf and NaN) -> fp64.
+
+    Normal: (-1)^s 2^(e-15) (1 + m/4); subnormal (e = 0): (-1)^s 2^-14 m/4.
+    """
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 2) & 0x1F
+    m = (c & 0x3).astype(np.float64)
+    mag = np.where(e == 0, m / 4.0 * 2.0 ** -14, (1.0 + m / 4.0) * np.exp2((e - 15).astype(np.float64)))
+    mag = np.where(e == 31, np.where(m == 0, np.inf, np.nan), mag)
+    return s * mag
+
+
+def _e5m2_finite_values():
+    """All 124 non-negative finite E5M2 values with their codes, exact."""
+    out = []
+    for code in range(0x7C):
+        e, m = code >> 2, code & 3
+        v = Fraction(m, 4) * Fraction(1, 2 ** 14) if e == 0 else (1 + Fraction(m, 4)) * Fraction(2) ** (e - 15)
+        out.append((v, code))
+    return out
+
+
+_E5M2_TABLE = _e5m2_finite_values()
+
+
+def e5m2_encode_exact(x: float) -> int:
+    """Scalar E5M2 encoder in exact rationals: nearest value, ties to the even
+    code, saturating to +-57344 (satfinite); NaN encodes as 0x7F."""
+    if math.isnan(x):
+        return 0x7F
+    sign = 0x80 if math.copysign(1.0, x) < 0 else 0
+    if math.isinf(x):
+        return sign | 0x7B
+    a = Fraction(abs(x))
+    if a >= Fraction(int(E5M2_MAX)):
+        return sign | 0x7B
+    best = None
+    for v, code in _E5M2_TABLE:
+        d = abs(a - v)
+        if best is None or d < best[0] or (d == best[0] and (code & 1) == 0):
+            best = (d, code)
+    return sign | best[1]
+
+
+def e5m2_encode(x: np.ndarray) -> np.ndarray:
+    """Vectorised E5M2 encoder (same rule as :func:`e5m2_encode_exact`): the
+    spacing around |x| is 2^(E-2) in normal binades (E >= -14) and 2^-16
+    below; np.rint rounds half to even."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    sign = np.where(np.signbit(x), 0x80, 0).astype(np.int64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        _, ex = np.frexp(a)
+        E = np.maximum(ex.astype(np.int64) - 1, -14)
+        quantum = np.exp2((E - 2).astype(np.float64))
+        n = np.rint(a / quantum)
+        v = n * quantum
+    v = np.where(np.isfinite(v), v, E5M2_MAX)
+    v = np.minimum(v, E5M2_MAX)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        _, ev = np.frexp(v)
+        Ev = ev.astype(np.int64) - 1
+        sub = v < 2.0 ** -14
+        code_sub = np.rint(v / 2.0 ** -16)
+        mant = np.rint((v / np.exp2(Ev.astype(np.float64)) - 1.0) * 4.0)
+        code_norm = ((Ev + 15) << 2) + mant.astype(np.int64)
+    code = np.where(sub, code_sub.astype(np.int64), code_norm)
+    code = np.where(v == 0, 0, code)
+    code = (sign | code).astype(np.uint8)
+    return np.where(np.isnan(x), np.uint8(0x7F), code).astype(np.uint8)
+
+
+# scale codec -> (largest finite value, encoder, decoder)
+SCALE_CODECS = {"e4m3": (E4M3_MAX, e4m3_encode, e4m3_decode), "e5m2": (E5M2_MAX, e5m2_encode, e5m2_decode)}
+
+
+# ---------------------------------------------------------------------------
 # Quantiser ("The idea": blocks of 64, 32-bit scale per block, scales
 # quantised again to 8 bits; inferensys: block-wise absmax, 8-bit floats).
 # ---------------------------------------------------------------------------
@@ -294,9 +381,10 @@ def _check_shape(N: int, K: int):
         raise ValueError("W must be [N, K] with K a multiple of 64")
 
 
-def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16, fmt: str = "nf4"):
+def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16, fmt: str = "nf4", scale: str = "e4m3"):
     """NF4 double quantisation of a bf16 weight ``[N, K]`` (``fmt`` swaps the
-    16 levels for one of the compared formats, see :func:`codebook`).
+    16 levels for one of the compared formats, see :func:`codebook`;
+    ``scale="e5m2"`` stores c2 as E5M2 with c1 = RN32(max / 57344)).
 
     Returns ``(codes, c2, c1)``:
       * ``codes`` uint8 ``[N*K/2]``: element 2j in the low nibble, 2j+1 in the
@@ -335,25 +423,27 @@ def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16, fmt: str = "nf4"):
     G = (nb + DQ_BLOCK - 1) // DQ_BLOCK
     c1 = np.empty(G, dtype=np.float32)
     c2 = np.empty(nb, dtype=np.uint8)
+    smax, encode, _ = SCALE_CODECS[scale]
     for g in range(G):
         cg = absmax[g * DQ_BLOCK:(g + 1) * DQ_BLOCK]
-        c1g = np.float32(cg.max()) / np.float32(E4M3_MAX)   # fp32 division
+        c1g = np.float32(cg.max()) / np.float32(smax)       # fp32 division
         c1[g] = c1g
         if c1g > 0:
-            c2[g * DQ_BLOCK:(g + 1) * DQ_BLOCK] = e4m3_encode((cg / c1g).astype(np.float32))
+            c2[g * DQ_BLOCK:(g + 1) * DQ_BLOCK] = encode((cg / c1g).astype(np.float32))
         else:
             c2[g * DQ_BLOCK:(g + 1) * DQ_BLOCK] = 0
     return codes.reshape(-1), c2, c1
 
 
-def decoded_scales(c2: np.ndarray, c1: np.ndarray) -> np.ndarray:
+def decoded_scales(c2: np.ndarray, c1: np.ndarray, scale: str = "e4m3") -> np.ndarray:
     """c^_b = RN32(dec(c2_b) * c1_g): the 32-bit scale used by the dequantiser."""
-    dec = e4m3_decode(c2).astype(np.float32)            # every E4M3 value is exact in fp32
+    dec = SCALE_CODECS[scale][2](c2).astype(np.float32)  # every 8-bit float value is exact in fp32
     g = np.arange(len(c2)) // DQ_BLOCK
     return (dec * c1[g]).astype(np.float32)             # fp32 multiply
 
 
-def dequant(codes: np.ndarray, c2: np.ndarray, c1: np.ndarray, N: int, K: int, fmt: str = "nf4") -> np.ndarray:
+def dequant(codes: np.ndarray, c2: np.ndarray, c1: np.ndarray, N: int, K: int, fmt: str = "nf4",
+            scale: str = "e4m3") -> np.ndarray:
     """doubleDequant(c1, c2, W_NF4) -> bf16 bits ``[N, K]`` (``fmt``: the
     levels the codes index, see :func:`codebook`).
 
@@ -367,7 +457,7 @@ def dequant(codes: np.ndarray, c2: np.ndarray, c1: np.ndarray, N: int, K: int, f
     code = np.empty((cb.shape[0], BLOCK), dtype=np.uint8)
     code[:, 0::2] = cb & 0xF
     code[:, 1::2] = cb >> 4
-    chat = decoded_scales(c2, c1)
+    chat = decoded_scales(c2, c1, scale)
     w = (q[code] * chat[:, None]).astype(np.float32)    # fp32 multiply
     return f32_to_bf16_bits(w).reshape(N, K)
 

@@ -106,14 +106,14 @@ def test_compared_format_levels_match_oracle_bitwise(q):
 
 
 def test_format_checks_before_any_launch(q):
-    """An unknown format or a nonzero reserved field is rejected on the host
+    """An unknown format or scale codec is rejected on the host
     (the fake pointers would fault if a kernel were launched)."""
     L = q.lib()
     P = ctypes.c_void_p
     fake = P(0x10000)
     arr = (ctypes.c_float * 16)()
     assert L.qlora_code_levels(3, arr) == -11 and L.qlora_code_levels(-1, arr) == -11
-    for fmt, res in ((3, 0), (0, 1)):
+    for fmt, res in ((3, 0), (0, 2), (0, -1)):
         w = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 128, fmt, res)
         assert L.qlora_nf4_quantize(fake, 64, 128, ctypes.byref(w), None, None) == -11
         assert L.qlora_nf4_dequant(ctypes.byref(w), fake, None, None) == -11

@@ -38,10 +38,10 @@ def make_case(M, N, K, r, seed, regime="config", zero_W=False, zero_L2=False):
     return X, W, L1, L2, dY
 
 
-def run_gpu(q, X, W, L1, L2, dY, s, backward=True, fmt="nf4"):
+def run_gpu(q, X, W, L1, L2, dY, s, backward=True, fmt="nf4", scale="e4m3"):
     tX, tW, tL1, tL2 = (from_bits(a) for a in (X, W, L1, L2))
     q.read_status()
-    w = q.quantize(tW, fmt=fmt)
+    w = q.quantize(tW, fmt=fmt, scale=scale)
     Y, T = q.linear_fwd(tX, w, tL1, tL2, s)
     out = {"Y": Y, "T": T}
     if backward:
@@ -52,9 +52,9 @@ def run_gpu(q, X, W, L1, L2, dY, s, backward=True, fmt="nf4"):
     return {k: to_f64(v) for k, v in out.items()}
 
 
-def oracle_ref(X, W, L1, L2, dY, s, backward=True, fmt="nf4"):
+def oracle_ref(X, W, L1, L2, dY, s, backward=True, fmt="nf4", scale="e4m3"):
     N, K = W.shape
-    What = O.bf16_bits_to_f64(O.dequant(*O.quantize(W, fmt=fmt), N, K, fmt=fmt))
+    What = O.bf16_bits_to_f64(O.dequant(*O.quantize(W, fmt=fmt, scale=scale), N, K, fmt=fmt, scale=scale))
     X64, L164, L264 = (O.bf16_bits_to_f64(a) for a in (X, L1, L2))
     Y, T = O.linear_fwd(X64, What, L164, L264, s)
     ref = {"Y": Y, "T": T}
@@ -105,23 +105,24 @@ def test_pair_forward_parity(lib, monkeypatch, M, N, K, r, pair):
         assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} pair={pair}")
 
 
-# The compared 4-bit formats through every kernel that dequantises on chip:
+# The compared 4-bit formats and the E5M2 scale codec through every kernel
+# that dequantises on chip:
 # the forward and dX engines (with a split reduction and without), the
 # few-token GEMV path and the opt-in CTA-pair forward.
 FORMAT_SHAPES = [(300, 256, 192, 16, "0"), (2048, 4096, 512, 32, "1"), (7, 1000, 704, 32, "0")]
 
 
-@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+@pytest.mark.parametrize("fmt,scale", [("fp4", "e4m3"), ("int4", "e4m3"), ("nf4", "e5m2"), ("int4", "e5m2")])
 @pytest.mark.parametrize("M,N,K,r,pair", FORMAT_SHAPES)
-def test_formats_linear_parity(lib, monkeypatch, fmt, M, N, K, r, pair):
+def test_formats_linear_parity(lib, monkeypatch, fmt, scale, M, N, K, r, pair):
     monkeypatch.setenv("QLORA_NF4_PAIR", pair)
     s = 0.75
     case = make_case(M, N, K, r, seed=M * 17 + N + K + r, regime="lora_heavy")
     backward = pair == "0"
-    got = run_gpu(lib, *case, s, backward=backward, fmt=fmt)
-    ref = oracle_ref(*case, s, backward=backward, fmt=fmt)
+    got = run_gpu(lib, *case, s, backward=backward, fmt=fmt, scale=scale)
+    ref = oracle_ref(*case, s, backward=backward, fmt=fmt, scale=scale)
     for k in got:
-        assert_close(got[k], ref[k], f"{k} {fmt} M={M} N={N} K={K} r={r} pair={pair}")
+        assert_close(got[k], ref[k], f"{k} {fmt}/{scale} M={M} N={N} K={K} r={r} pair={pair}")
 
 
 # Few-token forward (M <= 16, the weight-streaming stream-K GEMV path): one

@@ -13,10 +13,10 @@ from bit_nf4_quantized_15_b200 import workloads as WL
 pytestmark = pytest.mark.gpu
 
 
-def gpu_quant(q, Wb, fmt="nf4"):
+def gpu_quant(q, Wb, fmt="nf4", scale="e4m3"):
     W = from_bits(Wb)
     q.read_status()
-    w = q.quantize(W, fmt=fmt)
+    w = q.quantize(W, fmt=fmt, scale=scale)
     torch.cuda.synchronize()
     assert q.read_status() == 0
     return w
@@ -178,3 +178,22 @@ def test_formats_special_blocks(lib, fmt):
     w = gpu_quant(lib, Wb, fmt)
     assert_quant_equal(w, ref)
     assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, 6, 64, fmt=fmt))
+
+
+# ------------------------------------ scale codec variant: c2 stored as E5M2
+@pytest.mark.parametrize("fmt", ["nf4", "fp4"])
+@pytest.mark.parametrize("N,K,seed", [(3, 128, 20), (37, 64 * 300, 21), (256, 4096, 22)])
+def test_e5m2_scales_quantize_dequant_bitexact(lib, fmt, N, K, seed):
+    Wb = mixed_weights(N, K, seed)
+    ref = O.quantize(Wb, fmt=fmt, scale="e5m2")
+    w = gpu_quant(lib, Wb, fmt, "e5m2")
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, N, K, fmt=fmt, scale="e5m2"))
+
+
+def test_e5m2_scales_every_significand_pair(lib):
+    Wb = mantissa_pair_matrix()
+    ref = O.quantize(Wb, scale="e5m2")
+    w = gpu_quant(lib, Wb, "nf4", "e5m2")
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, *Wb.shape, scale="e5m2"))

@@ -111,3 +111,59 @@ def test_e4m3_encode_special():
     assert enc(2.0 ** -10) == 0x00     # tie between 0 and 2^-9: even code 0
     assert enc(3 * 2.0 ** -10) == 0x02 # tie between 1 and 2 (x 2^-9): even
     assert enc(-1.0) == 0x80 | 0x38
+
+
+# ------------------------------------------------------------------ E5M2
+# The scale-codec variant of the double quantisation (c2 as E5M2).
+def test_e5m2_decode_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e5m2).double().numpy()
+    ours = O.e5m2_decode(codes)
+    both_nan = np.isnan(ref) & np.isnan(ours)
+    assert np.all(both_nan | (ref == ours))
+
+
+def _e5m2_ties_and_neighbours():
+    vals = np.sort(O.e5m2_decode(np.arange(0x7C, dtype=np.uint8)))
+    mids = (vals[:-1] + vals[1:]) / 2
+    pts = np.concatenate([vals, mids, [61440.0, 65536.0, 1e6]]).astype(np.float32)
+    out = []
+    for p in pts:
+        out += [p, np.nextafter(p, np.float32(np.inf)), np.nextafter(p, np.float32(0))]
+    return np.array(out, dtype=np.float32)
+
+
+def test_e5m2_encode_matches_exact_on_ties():
+    x = _e5m2_ties_and_neighbours()
+    x = np.concatenate([x, -x])
+    fast = O.e5m2_encode(x)
+    slow = np.array([O.e5m2_encode_exact(float(v)) for v in x], dtype=np.uint8)
+    assert np.array_equal(fast, slow)
+
+
+def test_e5m2_encode_matches_exact_random():
+    rng = np.random.default_rng(12)
+    x = np.concatenate([rng.uniform(0, 60000, 10000), np.exp2(rng.uniform(-18, 16, 10000))]).astype(np.float32)
+    fast = O.e5m2_encode(x)
+    slow = np.array([O.e5m2_encode_exact(float(v)) for v in x], dtype=np.uint8)
+    assert np.array_equal(fast, slow)
+
+
+def test_e5m2_encode_matches_torch_in_range():
+    rng = np.random.default_rng(13)
+    x = np.concatenate([_e5m2_ties_and_neighbours(), rng.uniform(0, 57344, 100000).astype(np.float32),
+                        np.exp2(rng.uniform(-18, 15.8, 100000)).astype(np.float32)])
+    x = x[np.abs(x) <= 57344]
+    ref = torch.from_numpy(x.copy()).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(O.e5m2_encode(x), ref)
+
+
+def test_e5m2_encode_special():
+    enc = lambda v: int(O.e5m2_encode(np.array([v], dtype=np.float32))[0])
+    assert enc(0.0) == 0x00
+    assert enc(57344.0) == 0x7B
+    assert enc(61440.0) == 0x7B        # beyond the largest finite value: satfinite
+    assert enc(float("inf")) == 0x7B
+    assert enc(float("nan")) == 0x7F
+    assert enc(2.0 ** -17) == 0x00     # tie between 0 and 2^-16: even code 0
+    assert enc(1.0) == 0x3C and enc(-1.0) == 0xBC

@@ -140,3 +140,32 @@ def test_nf4_beats_the_compared_formats_on_normal_weights():
         What = O.bf16_bits_to_f64(O.dequant(*O.quantize(W, fmt=f), N, K, fmt=f))
         err[f] = float(np.mean((w - What) ** 2))
     assert err["nf4"] < err["fp4"] and err["nf4"] < err["int4"]
+
+
+# ------------------------------------------------ scale codec: E5M2 for c2
+@pytest.mark.parametrize("fmt", ["nf4", "fp4"])
+@pytest.mark.parametrize("case", range(3))
+def test_e5m2_scales_match_bruteforce(fmt, case):
+    W = _tiny_inputs()[case]
+    N, K = W.shape
+    a = O.quantize(W, fmt=fmt, scale="e5m2")
+    b = brute_quantize(W, O.codebook(fmt), scale="e5m2")
+    for x, y in zip(a, b):
+        assert np.array_equal(np.asarray(x).view(np.uint8), np.asarray(y).view(np.uint8))
+    assert np.array_equal(O.dequant(*a, N, K, fmt=fmt, scale="e5m2"),
+                          brute_dequant(*a, N, K, O.codebook(fmt), scale="e5m2"))
+
+
+def test_e5m2_scale_bounds():
+    """Two mantissa bits: relative scale error <= 2^-3 in E5M2's normal range;
+    the codes do not depend on the scale codec."""
+    rng = np.random.default_rng(17)
+    W = _bf16(rng.standard_t(3, (256, 64 * 64)) * 0.02)
+    codes, c2, c1 = O.quantize(W, scale="e5m2")
+    assert np.array_equal(codes, O.quantize(W)[0])
+    c = O.block_absmax(W).astype(np.float64)
+    chat = O.decoded_scales(c2, c1, "e5m2").astype(np.float64)
+    c1r = np.repeat(c1.astype(np.float64), 256)[: len(c)]
+    assert np.all(O.e5m2_decode(c2) <= 57344.0)
+    normal = c / c1r >= 2.0 ** -14
+    assert (np.abs(chat - c)[normal] / c[normal]).max() <= 2.0 ** -3 + 1e-6

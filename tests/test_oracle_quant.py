@@ -65,11 +65,26 @@ def e4m3_nearest(a: Fraction) -> int:
     return best[1]
 
 
+_E5M2 = []
+for _c in range(0x7C):
+    _e, _m = _c >> 2, _c & 3
+    _E5M2.append(((Fraction(_m, 4) / 2 ** 14) if _e == 0 else (1 + Fraction(_m, 4)) * Fraction(2) ** (_e - 15), _c))
+
+
+def e5m2_nearest(a: Fraction) -> int:
+    """Non-negative rational -> E5M2 code: nearest value, ties to even code,
+    anything at or above 57344 saturates."""
+    if a >= 57344:
+        return 0x7B
+    best = min(_E5M2, key=lambda vc: (abs(a - vc[0]), vc[1] & 1))
+    return best[1]
+
+
 def bf16_value(bits: int) -> Fraction:
     return Fraction(float(O.bf16_bits_to_f32(np.array([bits], np.uint16))[0]))
 
 
-def brute_quantize(W_bits: np.ndarray, levels=None):
+def brute_quantize(W_bits: np.ndarray, levels=None, scale="e4m3"):
     q = [Fraction(float(v)) for v in (O.nf4_codebook() if levels is None else levels)]
     mids = [(q[i] + q[i + 1]) / 2 for i in range(15)]
     flat = W_bits.reshape(-1).tolist()
@@ -87,17 +102,18 @@ def brute_quantize(W_bits: np.ndarray, levels=None):
             codes[idx // 2] |= code << (4 * (idx & 1))
     G = (nb + 255) // 256
     c1, c2 = [], []
+    smax, nearest = (448, e4m3_nearest) if scale == "e4m3" else (57344, e5m2_nearest)
     for g in range(G):
         grp = absmax[256 * g:256 * g + 256]
-        c1g = rn32(max(grp) / 448)
+        c1g = rn32(max(grp) / smax)
         c1.append(c1g)
         for c in grp:
-            c2.append(0 if c1g == 0 else e4m3_nearest(rn32(c / c1g)))
+            c2.append(0 if c1g == 0 else nearest(rn32(c / c1g)))
     return (np.frombuffer(bytes(codes), np.uint8), np.array(c2, np.uint8),
             np.array([float(v) for v in c1], np.float32))
 
 
-def brute_dequant(codes, c2, c1, N, K, levels=None):
+def brute_dequant(codes, c2, c1, N, K, levels=None, scale="e4m3"):
     q = [Fraction(float(v)) for v in (O.nf4_codebook() if levels is None else levels)]
     out = np.empty(N * K, np.uint16)
     for idx in range(N * K):
@@ -105,8 +121,12 @@ def brute_dequant(codes, c2, c1, N, K, levels=None):
         b = idx // 64
         dec = 0
         cc = int(c2[b])
-        e, m = (cc >> 3) & 15, cc & 7
-        dec = (Fraction(m, 8) / 64) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+        if scale == "e4m3":
+            e, m = (cc >> 3) & 15, cc & 7
+            dec = (Fraction(m, 8) / 64) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+        else:
+            e, m = (cc >> 2) & 31, cc & 3
+            dec = (Fraction(m, 4) / 2 ** 14) if e == 0 else (1 + Fraction(m, 4)) * Fraction(2) ** (e - 15)
         chat = rn32(dec * Fraction(float(c1[b // 256])))
         v = rnbf16(rn32(q[code] * chat))
         out[idx] = O.f32_to_bf16_bits(np.array([float(v)], np.float32))[0]
