@@ -261,6 +261,34 @@ def gemv_rates(q, WL, dev, hbm_gbs, pk_kind, copies=4, reps=20):
     return res
 
 
+def bf16_gemm_ms(q, layers, reps):
+    """Mean device time per step of the two weight products of every linear,
+    Y = X.W^T and dX = dY.W, done by torch.matmul (cuBLAS) on the dequantised
+    bf16 weight: the 16-bit baseline the pages compare QLoRA's
+    dequantise-on-the-fly with ("roughly 30-40% slower")."""
+    import torch
+    Wh = [q.dequant(L["w"]) for L in layers]
+    outs = [(torch.empty_like(L["Y"]), torch.empty_like(L["dX"])) for L in layers]
+
+    def run():
+        for L, W, (Y, dX) in zip(layers, Wh, outs):
+            torch.matmul(L["X"], W.t(), out=Y)
+            torch.matmul(L["dY"], W, out=dX)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del Wh, outs
+    return ms
+
+
 # ------------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -358,6 +386,8 @@ def run_ours(args):
     gemm_flops = sum(main_gemm_flops(M, L["lin"].N, L["lin"].K, r) for L in layers)
     pk, pk_kind = peaks()
     achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
+    # context: the same products with a plain bf16 weight (cuBLAS)
+    bf16_ms = bf16_gemm_ms(q, layers, max(args.steps, 3))
 
     # ---- NF4 quantise / dequantise: the bulk round trip of 2^31 weights (4 GiB
     # of bf16: half N(0, 0.02), half Student-t(3) x 0.02 with x50 outliers),
@@ -452,6 +482,10 @@ def run_ours(args):
                          "traffic_unit": "bytes per launch (DRAM read + write, ncu, mean over the step's launches)",
                          "peak_source": f"{pk_kind} sustained dense bf16",
                          "launches_timed": 2 * n_lin, "ms_per_launch": gemm_ms / (2 * n_lin)},
+            "context_bf16_gemm": {
+                "what": "Y = X.W^T and dX = dY.W of the 7 linears per step: the fused dequant-GEMM launches (NF4 "
+                        "weight, LoRA term included) against torch.matmul (cuBLAS) on the dequantised bf16 weight",
+                "fused_ms_per_step": gemm_ms, "bf16_ms_per_step": bf16_ms, "fused_over_bf16": gemm_ms / bf16_ms},
             "quant": {"workload": RT_WORKLOAD, "value": quant_gbs, "unit": "GB/s", "frac": quant_gbs / hbm, "peak": hbm,
                       "bytes": qb, "peak_source": f"{pk_kind} HBM copy"},
             "dequant": {"workload": RT_WORKLOAD, "value": dequant_gbs, "unit": "GB/s", "frac": dequant_gbs / hbm, "peak": hbm,
