@@ -197,3 +197,16 @@ def test_e5m2_scales_every_significand_pair(lib):
     w = gpu_quant(lib, Wb, "nf4", "e5m2")
     assert_quant_equal(w, ref)
     assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, *Wb.shape, scale="e5m2"))
+
+
+def test_quantize_sharded_single_rank_equals_quantize(lib):
+    """The sharded quantiser's per-rank step (the library quantiser on a flat
+    [1, len] view of a run of whole 16384-weight groups) without a process
+    group: the whole weight as one share, bit-exact against the oracle."""
+    from bit_nf4_quantized_15_b200.sharded import quantize_sharded
+    Wb = mixed_weights(37, 64 * 300, 23)
+    w = quantize_sharded(from_bits(Wb))
+    torch.cuda.synchronize()
+    assert (w.N, w.K) == (37, 64 * 300)
+    assert_quant_equal(w, O.quantize(Wb))
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*O.quantize(Wb), 37, 64 * 300))
