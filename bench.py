@@ -112,7 +112,10 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        # the raw samples are kept for inspection: QLORA_CLOCKS_DIR, else the system temp directory
+        import tempfile
+        base = os.environ.get("QLORA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(base, f"clocks_bench_{os.getpid()}.csv")
 
     def start(self):
         try:
