@@ -169,3 +169,34 @@ def test_e5m2_scale_bounds():
     assert np.all(O.e5m2_decode(c2) <= 57344.0)
     normal = c / c1r >= 2.0 ** -14
     assert (np.abs(chat - c)[normal] / c[normal]).max() <= 2.0 ** -3 + 1e-6
+
+
+# ------------------------------------------ planted mistakes (CPU only)
+def test_planted_e5m2_with_e4m3_range_is_caught():
+    """E5M2 codes with the E4M3 divisor (448) for c1: the brute-force pin
+    (57344) rejects it."""
+    W = _tiny_inputs()[1]
+    codes, _, _ = O.quantize(W, scale="e5m2")
+    absmax = O.block_absmax(W)
+    c1_bad = np.array([np.float32(absmax[g * 256:(g + 1) * 256].max()) / np.float32(448.0)
+                       for g in range((len(absmax) + 255) // 256)], np.float32)
+    ref = brute_quantize(W, O.codebook("nf4"), scale="e5m2")
+    assert not np.array_equal(c1_bad.view(np.uint32), ref[2].view(np.uint32))
+
+
+def test_planted_fp4_pad_at_the_top_is_caught():
+    """The FP4 table with its pad level above +1 instead of below -1 fails
+    the E2M1 level pin and changes the codes of the tiny cases."""
+    good = O.codebook("fp4")
+    bad = np.concatenate([good[1:], np.array([2.0], np.float32)])
+    vals = sorted({_e2m1_value(b) for b in range(16)})
+    want = np.array([_as_f32(rn32(v / 6)) for v in vals], np.float32)
+    assert np.array_equal(good[1:], want) and not np.array_equal(bad[1:], want)
+    W = _tiny_inputs()[0]
+    assert not np.array_equal(brute_quantize(W, bad)[0], O.quantize(W, fmt="fp4")[0])
+
+
+def test_planted_int4_over_8_is_caught():
+    """Levels k/8 instead of k/7 (an asymmetric int4 reading) fail the pin."""
+    bad = np.array([np.float32(k / 8) for k in range(-8, 8)], np.float32)
+    assert not np.array_equal(bad, O.codebook("int4"))
