@@ -22,7 +22,8 @@ import torch
 
 __all__ = [
     "lib", "NF4Weight", "quantize", "quantize_into", "dequant", "workspace_bytes", "linear_fwd", "linear_bwd",
-    "codebook", "FORMATS", "SCALES", "status_string", "kernel_launches", "set_gemm_events", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
+    "codebook", "FORMATS", "SCALES", "status_string", "kernel_launches", "set_gemm_events",
+    "debug_stall_next_gemm", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
@@ -68,6 +69,7 @@ _SIGS = {
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_kernel_launches": (ctypes.c_uint64, []),
     "qlora_set_gemm_events": (ctypes.c_int, [_P, _P]),
+    "qlora_debug_stall_next_gemm": (ctypes.c_int, [ctypes.c_uint64]),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P, ctypes.c_int,
                                                 ctypes.c_float, _P, _P, _P, _P]),
 }
@@ -100,6 +102,13 @@ def set_gemm_events(ev_start, ev_end):
     h0 = None if ev_start is None else ctypes.c_void_p(ev_start.cuda_event)
     h1 = None if ev_end is None else ctypes.c_void_p(ev_end.cuda_event)
     _check(lib().qlora_set_gemm_events(h0, h1))
+
+
+def debug_stall_next_gemm(wait_ns: int):
+    """Failure-detection test hook: the next fused dequant-GEMM launch issues
+    no loads and bounds its waits by `wait_ns`, so they expire and the device
+    status word reads QLORA_ERR_TIMEOUT (see qlora_debug_stall_next_gemm)."""
+    _check(lib().qlora_debug_stall_next_gemm(int(wait_ns)))
 
 
 def status_string(code: int) -> str:

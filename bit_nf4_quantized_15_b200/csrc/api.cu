@@ -139,17 +139,26 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Diagnostic events around the fused dequant-GEMM (qlora_set_gemm_events).
 cudaEvent_t g_ev_start = nullptr, g_ev_end = nullptr;
+// Failure-detection hook (qlora_debug_stall_next_gemm): wait bound of the
+// next fused dequant-GEMM launch, whose producer then issues no loads.
+uint64_t g_stall_ns = 0;
 
 int run_timed(EngineArgs& a, int amode, const GemmPlan& p, float* partial, cudaStream_t st) {
   cudaEvent_t e0 = g_ev_start, e1 = g_ev_end;
   g_ev_start = g_ev_end = nullptr;
+  const uint64_t stall_ns = g_stall_ns;
+  g_stall_ns = 0;
+  if (stall_ns && amode != A_PAIR_K) {
+    a.stall = 1;
+    a.wait_ns = stall_ns;
+  }
   if (e0 && cudaEventRecord(e0, st) != cudaSuccess) return QLORA_ERR_CUDA;
   const int rc = run(a, amode, p, partial, st);
   if (rc == QLORA_OK && e1 && cudaEventRecord(e1, st) != cudaSuccess) return QLORA_ERR_CUDA;
   return rc;
 }
 
-bool valid_rank(int r) { return r >= 16 && r <= 128 && r % 16 == 0; }
+bool valid_rank(int r) { return r >= 8 && r <= 128 && r % 8 == 0; }
 
 // Workspace layout shared by the forward and the backward:
 //   [0]             bf16 s.T   [M][r]
@@ -200,7 +209,7 @@ const char* qlora_status_string(int code) {
     case QLORA_ERR_NULL: return "a required pointer is NULL";
     case QLORA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
     case QLORA_ERR_SHAPE: return "invalid shape (need K % 64 == 0, N % 8 == 0, sizes >= 1)";
-    case QLORA_ERR_RANK: return "unsupported LoRA rank (need r % 16 == 0, 16 <= r <= 128)";
+    case QLORA_ERR_RANK: return "unsupported LoRA rank (need r % 8 == 0, 8 <= r <= 128)";
     case QLORA_ERR_WORKSPACE: return "workspace too small";
     case QLORA_ERR_CUDA: return "CUDA runtime or driver call failed";
     case QLORA_ERR_NONFINITE: return "weight holds an Inf or NaN";
@@ -222,6 +231,11 @@ int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes, size_t* c
 }
 
 uint64_t qlora_kernel_launches(void) { return launches_so_far(); }
+
+int qlora_debug_stall_next_gemm(uint64_t wait_ns) {
+  g_stall_ns = wait_ns;
+  return QLORA_OK;
+}
 
 int qlora_set_gemm_events(void* ev_start, void* ev_end) {
   g_ev_start = (ev_start && ev_end) ? reinterpret_cast<cudaEvent_t>(ev_start) : nullptr;

@@ -64,7 +64,9 @@ QDEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // false (after flagging the CTA and the caller's status) on timeout or when
 // another role of the CTA has already aborted.  Plain polling: a suspended
 // wait (try_wait with a time hint) was measured to wake up late.
-QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+// `limit_ns` is the bound (QNF4_WAIT_NS unless a launch asks for less).
+QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                    uint64_t limit_ns = QNF4_WAIT_NS) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -72,7 +74,7 @@ QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, in
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 63) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > QNF4_WAIT_NS) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         report(status, QLORA_ERR_TIMEOUT);
         return false;

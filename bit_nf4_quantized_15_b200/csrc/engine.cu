@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
   // block holding both.
   const int ext_iters = z == 0 && args.kb_ext ? (AMODE == A_DEQ_K ? 1 + args.kb_ext : args.kb_ext) : 0;
   const int n_iters = my_kb + ext_iters;
+  const uint64_t lim = args.wait_ns ? args.wait_ns : QNF4_WAIT_NS;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -121,11 +122,11 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !args.stall) {
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status)) break;
+        if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status, lim)) break;
         uint8_t* sa = smem + s * L::STAGE;
         uint8_t* sb = sa + kA;
         uint8_t* sc = sb + L::B;
@@ -167,8 +168,8 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const bool ext = it >= my_kb;
-        bool ok = mbar_wait(full + s, ph, abort_flag, args.status);
-        if (ok && AMODE != A_TMA && !ext) ok = mbar_wait(afull + s, ph, abort_flag, args.status);
+        bool ok = mbar_wait(full + s, ph, abort_flag, args.status, lim);
+        if (ok && AMODE != A_TMA && !ext) ok = mbar_wait(afull + s, ph, abort_flag, args.status, lim);
         if (!ok) break;
         tc_fence_after();
         const uint8_t* sa = smem + s * L::STAGE;
@@ -246,9 +247,9 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
           c1v = __ldg(args.c1 + (f >> 8));
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
-        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane)) break;
+        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane, lim)) break;
         tc_fence_after();
-        if (!warp_wait(full + s, ph, abort_flag, args.status, lane)) break;
+        if (!warp_wait(full + s, ph, abort_flag, args.status, lane, lim)) break;
         const uint4 c0 = *reinterpret_cast<const uint4*>(ctile + (sw << 4));
         const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + ((sw ^ 1) << 4));
         uint32_t o[16];
@@ -306,8 +307,8 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
           }
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
-        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane)) break;
-        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane)) break;
+        if (!warp_wait(empty + grp, ph ^ 1u, abort_flag, args.status, lane, lim)) break;
+        if (!warp_wait(full + grp, ph, abort_flag, args.status, lane, lim)) break;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint4 cw = *reinterpret_cast<const uint4*>(ctile + (((2 * mb + h) ^ swz) << 4));
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
     // ------------------------------------------------------------ epilogue
     // G warps per lane quarter: group grp stores the 16-column chunks
     // grp, grp + G, ... of the tile.
-    const bool ok = warp_wait(accum, 0, abort_flag, args.status, lane);
+    const bool ok = warp_wait(accum, 0, abort_flag, args.status, lane, lim);
     tc_fence_after();
     const int64_t row = row0 + q4 * 32 + lane;
     const EpiArgs& e = args.epi;

@@ -42,9 +42,10 @@ QDEV void epi_store(const EpiArgs& e, int64_t row, int64_t col, float v) {
 
 // Warp-wide wait: lane 0 polls (bounded), then every lane takes one
 // acquiring look at the completed phase.
-QDEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status, int lane) {
+QDEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status, int lane,
+                    uint64_t limit_ns = QNF4_WAIT_NS) {
   int ok = 1;
-  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status, limit_ns) ? 1 : 0;
   ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
   if (ok) mbar_try_wait(smem_u32(bar), parity);
   return ok != 0;

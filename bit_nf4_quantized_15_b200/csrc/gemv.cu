@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
   const int64_t n0 = (int64_t)blockIdx.x * 32, n = n0 + lane;
   const int rt = (int)(n0 / 128), rl = (int)(n % 128);
   const bool valid = n < N;
-  const int rq = r / 4, j0 = w * rq;  // this warp's adapter columns (r/4 is a multiple of 4)
+  const int rq = r / 4, j0 = w * rq;  // this warp's adapter columns (r % 8 == 0, so rq is even)
   // L2 first: it does not depend on the previous kernels
   float l2v[32];
 #pragma unroll
@@ -492,16 +492,14 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
   }
   __syncthreads();
 #pragma unroll
-  for (int q4 = 0; q4 < 8; ++q4) {
-    if (q4 * 4 < rq) {
+  for (int q2 = 0; q2 < 16; ++q2) {
+    if (q2 * 2 < rq) {  // j0 + 2 q2 is even: 8-byte aligned pairs of s.T
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
         if (m < M) {
-          const float4 s4 = *reinterpret_cast<const float4*>(sT + m * 128 + j0 + q4 * 4);
-          acc[m] = __fmaf_rn(s4.x, l2v[q4 * 4 + 0], acc[m]);
-          acc[m] = __fmaf_rn(s4.y, l2v[q4 * 4 + 1], acc[m]);
-          acc[m] = __fmaf_rn(s4.z, l2v[q4 * 4 + 2], acc[m]);
-          acc[m] = __fmaf_rn(s4.w, l2v[q4 * 4 + 3], acc[m]);
+          const float2 s2 = *reinterpret_cast<const float2*>(sT + m * 128 + j0 + q2 * 2);
+          acc[m] = __fmaf_rn(s2.x, l2v[q2 * 2 + 0], acc[m]);
+          acc[m] = __fmaf_rn(s2.y, l2v[q2 * 2 + 1], acc[m]);
         }
       }
     }

@@ -77,6 +77,8 @@ struct EngineArgs {
   float* partial;    // [splits][cols][rows] fp32 when splits > 1
   EpiArgs epi;
   int* status;
+  uint64_t wait_ns;  // bound of every internal wait (0: the default, 4 s)
+  int stall;         // failure-detection hook: the producer issues no loads
   float q[16];
 };
 

@@ -50,7 +50,7 @@ enum {
   QLORA_ERR_NULL = -1,        /* a required pointer is NULL */
   QLORA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
   QLORA_ERR_SHAPE = -3,       /* K % 64 != 0, N % 8 != 0, a size < 1 or too large */
-  QLORA_ERR_RANK = -4,        /* r not a multiple of 16 in [16, 128] */
+  QLORA_ERR_RANK = -4,        /* r not a multiple of 8 in [8, 128] */
   QLORA_ERR_WORKSPACE = -5,   /* ws too small (see qlora_workspace_bytes) */
   QLORA_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
   QLORA_ERR_NONFINITE = -7,   /* device status: W holds an Inf or NaN */
@@ -168,7 +168,7 @@ QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  *   X   : bf16[M][K]     L1 : bf16[K][r]     L2 : bf16[r][N]
  *   Y   : bf16[M][N]     T_save : float[M][r]
  *   ws  : device workspace of ws_bytes >= qlora_workspace_bytes(M, N, K, r)
- * Requires K % 64 == 0, N % 8 == 0, r % 16 == 0 and 16 <= r <= 128.
+ * Requires K % 64 == 0, N % 8 == 0, r % 8 == 0 and 8 <= r <= 128.
  * With QLORA_NF4_PAIR=1 in the environment (read at each call), grids of at
  * least one 128 x 256 tile per SM run on the CTA-pair kernel (cta_group::2)
  * instead of the single-CTA one: same result within the same tolerance.
@@ -208,8 +208,9 @@ QLORA_API int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M,
  * that loads it, held until exit.  A problem whose qlora_workspace_bytes()
  * exceeds 8 MiB is rejected with QLORA_ERR_SCRATCH_LIMIT before anything is
  * launched.  The first call on a device looks up the array's device address
- * (once per device, that device current); make that first call before any
- * stream capture.  All calls share the one array: calls that overlap on the
+ * (once per device, that device current; again after the device's context
+ * has been re-created, e.g. by cudaDeviceReset); make that first call before
+ * any stream capture.  All calls share the one array: calls that overlap on the
  * GPU race and must be serialised by the caller.  Allocates nothing.
  */
 QLORA_API int qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
@@ -223,6 +224,18 @@ QLORA_API int qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, const qlora
  * just after it (and after its split reduction, if any); the hook is then
  * cleared.  Process-wide, not thread-safe; NULL, NULL clears it. */
 QLORA_API int qlora_set_gemm_events(void* ev_start, void* ev_end);
+
+/* Failure-detection test hook (diagnostic; the method has no counterpart).
+ * The next fused dequant-GEMM launch of qlora_linear_fwd or qlora_linear_bwd
+ * (the Y launch of a forward with more than 16 tokens, resp. the dX launch
+ * of a backward; not the opt-in CTA-pair forward) runs with its TMA producer
+ * issuing no loads and every internal wait bounded by wait_ns nanoseconds
+ * instead of 4 s.  Its waits then expire: the kernel writes
+ * QLORA_ERR_TIMEOUT to *status_dev, frees its tensor memory and returns
+ * with nothing in flight, so the context stays usable; that call's outputs
+ * are unspecified.  One-shot and process-wide, not thread-safe; 0 cancels a
+ * pending request. */
+QLORA_API int qlora_debug_stall_next_gemm(uint64_t wait_ns);
 
 /* Number of kernels this process has launched through the library so far
  * (all devices, all calls).  A diagnostic for counting launches. */

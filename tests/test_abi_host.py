@@ -58,7 +58,7 @@ def test_storage_bytes(q):
 
 
 def test_status_strings(q):
-    for code in range(-9, 1):
+    for code in range(-11, 1):
         assert q.status_string(code)
     assert "unknown" in q.status_string(-99)
 
@@ -67,6 +67,10 @@ def test_workspace_bytes_host(q):
     L = q.lib()
     assert L.qlora_workspace_bytes(16, 4096, 4096, 16) > 0
     assert L.qlora_workspace_bytes(16, 4096, 4096, 17) == 0      # bad rank
+    assert L.qlora_workspace_bytes(16, 4096, 4096, 8) > 0        # r % 8 == 0 in [8, 128]
+    assert L.qlora_workspace_bytes(1000, 4096, 4096, 24) > 0
+    for bad in (0, 4, 12, 136, 256):
+        assert L.qlora_workspace_bytes(16, 4096, 4096, bad) == 0
     assert L.qlora_workspace_bytes(16, 4096, 100, 16) == 0       # K % 64
     assert L.qlora_workspace_bytes(16, 4100, 4096, 16) == 0      # N % 8
 

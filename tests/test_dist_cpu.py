@@ -1,7 +1,7 @@
 """Host logic of the multi-GPU path on the CPU: two gloo ranks run the
-bench's max-over-ranks timing reduction and the per-step all-reduce of the
-adapter gradients (the only exchange data parallelism needs: W is frozen and
-gets no gradient)."""
+bench's max-over-ranks timing reduction and the package's per-step
+all-reduce of the adapter gradients (the only exchange data parallelism
+needs: W is frozen and gets no gradient)."""
 
 import os
 import socket
@@ -28,21 +28,31 @@ def _worker(rank, world, port, q):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     import bench
+    from bit_nf4_quantized_15_b200.data_parallel import AdapterGrads
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         t_max = bench.max_over_ranks(10.0 + rank, world, "cpu")
-        # adapter gradients of 2 linears in one flat buffer, rank-dependent values
-        grads = torch.arange(12, dtype=torch.float32) * (rank + 1)
-        dL1 = grads[:8].view(4, 2)
-        dist.all_reduce(grads)
+        # the package's exchange: two linears' dL1/dL2 in one flat buffer,
+        # written through the per-linear views with rank-dependent values
+        g = AdapterGrads([(3, 2), (5, 4)], r=2, device="cpu")
+        for i, (N, K) in enumerate(g.shapes):
+            g.dL1[i].copy_(torch.arange(K * 2, dtype=torch.float32).view(K, 2) * (rank + 1) + i)
+            g.dL2[i].copy_(torch.arange(2 * N, dtype=torch.float32).view(2, N) * (rank + 1) - i)
+        g.all_reduce()
+        summed = [(g.dL1[i].clone(), g.dL2[i].clone()) for i in range(2)]
+        g.all_reduce(average=True)
         bench.barrier(world)
-        q.put((rank, t_max, grads.tolist(), dL1.sum().item()))
+        q.put((rank, t_max, g.flat.numel(), [(a.tolist(), b.tolist()) for a, b in summed],
+               [(a.tolist(), b.tolist()) for a, b in zip(g.dL1, g.dL2)]))
     finally:
         dist.destroy_process_group()
 
 
 def test_two_gloo_ranks_timing_and_grad_allreduce():
+    """Two gloo ranks: the bench's max-over-ranks timing, and the package's
+    adapter-gradient exchange (AdapterGrads.all_reduce) that the bench calls
+    once per step."""
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -53,11 +63,31 @@ def test_two_gloo_ranks_timing_and_grad_allreduce():
         p.join(120)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
-    expect = [float(i * 3) for i in range(12)]  # (1 + 2) * i
-    for rank, t_max, grads, view_sum in res:
+    expect_sum, expect_avg = [], []
+    for i, (N, K) in enumerate([(3, 2), (5, 4)]):
+        a = torch.arange(K * 2, dtype=torch.float32).view(K, 2)
+        b = torch.arange(2 * N, dtype=torch.float32).view(2, N)
+        s1, s2 = a * 3 + 2 * i, b * 3 - 2 * i        # (1 + 2) x + 2 i over the two ranks
+        expect_sum.append((s1.tolist(), s2.tolist()))
+        expect_avg.append(((s1 * 2 / 2).tolist(), (s2 * 2 / 2).tolist()))
+    for rank, t_max, n, summed, averaged in res:
         assert t_max == 11.0                     # the slowest rank's time
-        assert grads == expect                   # summed over ranks, same on every rank
-        assert view_sum == sum(expect[:8])       # views into the flat buffer see the reduced values
+        assert n == (2 * 2 + 2 * 3) + (4 * 2 + 2 * 5)
+        assert summed == expect_sum              # summed over ranks, same on every rank, seen through the views
+        assert averaged == expect_avg            # the second exchange sums the sums and divides by world
+
+
+def test_adapter_grads_single_process_is_a_noop():
+    sys.path.insert(0, ROOT)
+    from bit_nf4_quantized_15_b200.data_parallel import AdapterGrads, adapter_grad_elems
+    g = AdapterGrads([(8, 64), (16, 128)], r=4, device="cpu")
+    assert g.flat.numel() == adapter_grad_elems(8, 64, 4) + adapter_grad_elems(16, 128, 4)
+    assert g.dL1[1].shape == (128, 4) and g.dL2[1].shape == (4, 16)
+    g.dL2[0].fill_(3.0)
+    g.all_reduce()
+    assert g.flat[64 * 4:64 * 4 + 32].eq(3.0).all() and g.nbytes == g.flat.numel() * 4
+    with pytest.raises(ValueError):
+        adapter_grad_elems(0, 64, 4)
 
 
 def test_reference_arm_only_rank0_prints():

@@ -248,3 +248,35 @@ def test_full_llama65b_ffn_gemv(lib, M, which):
 def test_full_llama7b_block_linear(lib, which):
     wl = WL.WORKLOADS["llama7b_block"]
     _full_linear(lib, wl, wl.linears[which], seed=which)
+
+
+@pytest.mark.parametrize("which", [0, 4, 6])   # q (8192x8192), gate (22016x8192), down (8192x22016)
+def test_full_llama65b_block_linear(lib, which):
+    """The LLaMA-65B block at its full size: 8192 tokens, r = 64, alpha = 16,
+    W ~ N(0, 0.015), dY ~ N(0, 1e-2), in the launch configuration the bench
+    times (64 sampled rows of Y, T and dX against the fp64 oracle; dL1 and dL2
+    in full)."""
+    wl = WL.WORKLOADS["llama65b_block"]
+    _full_linear(lib, wl, wl.linears[which], seed=which)
+
+
+# Ranks that are multiples of 8 but not of 16 (r = 8, 24): the adapters are
+# narrower than one 16-wide MMA step and the TMA zero-fills the rest of the
+# 64-wide operand tiles; the few-token path's T slices and finish kernel see
+# odd per-warp column counts.  Engine (with and without split reductions),
+# few-token GEMV and the opt-in CTA-pair forward.
+RANK8_SHAPES = [(37, 136, 256, 8, "0"), (300, 1000, 640, 24, "0"), (1024, 1024, 2048, 8, "0"),
+                (5, 2056, 1536, 8, "0"), (16, 4096, 512, 24, "0"), (1000, 4736, 256, 8, "1")]
+
+
+@pytest.mark.parametrize("M,N,K,r,pair", RANK8_SHAPES)
+@pytest.mark.parametrize("regime", ["config", "lora_heavy"])
+def test_rank_multiple_of_8(lib, monkeypatch, M, N, K, r, pair, regime):
+    monkeypatch.setenv("QLORA_NF4_PAIR", pair)
+    s = 16.0 / r if regime == "config" else 0.75
+    case = make_case(M, N, K, r, seed=M * 19 + N + K + r, regime=regime)
+    backward = pair == "0"
+    got = run_gpu(lib, *case, s, backward=backward)
+    ref = oracle_ref(*case, s, backward=backward)
+    for k in got:
+        assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} pair={pair} {regime}")

@@ -330,3 +330,43 @@ def test_planted_tie_rule_is_caught():
         return (15 - np.argmin(d[..., ::-1], axis=-1)).astype(np.uint8)
 
     assert orig(m)[0] == 7 and up(m)[0] == 8
+
+
+def _three_groups():
+    """600 blocks = two full c1 groups of 256 and a partial third of 88, each
+    at its own magnitude (x1, x300, /500), so that a block or a scale read
+    from the wrong group changes c1, c2 or the dequantised weights."""
+    rng = np.random.default_rng(9)
+    a = rng.normal(0, 0.02, 600 * 64)
+    a[256 * 64:512 * 64] *= 300.0
+    a[512 * 64:] /= 500.0
+    return _bf16(a).reshape(25, 1536)
+
+
+def test_bruteforce_spans_groups_with_partial_last():
+    W = _three_groups()
+    N, K = W.shape
+    got = O.quantize(W)
+    ref = brute_quantize(W)
+    assert got[2].shape == (3,) and len(set(got[2].tolist())) == 3
+    for x, y in zip(got, ref):
+        assert np.array_equal(np.asarray(x).view(np.uint8), np.asarray(y).view(np.uint8))
+    assert np.array_equal(O.dequant(*got, N, K), brute_dequant(*ref, N, K))
+
+
+def test_planted_group_index_slip_is_caught():
+    """A dequantiser that takes c1 of block b from group b // 255 instead of
+    b // 256 disagrees with the brute-force dequantiser on the three-group
+    input."""
+    W = _three_groups()
+    N, K = W.shape
+    codes, c2, c1 = O.quantize(W)
+    dec = O.e4m3_decode(c2).astype(np.float32)
+    g = np.minimum(np.arange(len(c2)) // 255, len(c1) - 1)
+    chat = (dec * c1[g]).astype(np.float32)
+    q = O.nf4_codebook()
+    code = np.empty((len(c2), 64), np.uint8)
+    cb = codes.reshape(-1, 32)
+    code[:, 0::2], code[:, 1::2] = cb & 15, cb >> 4
+    slipped = O.f32_to_bf16_bits((q[code] * chat[:, None]).astype(np.float32)).reshape(N, K)
+    assert not np.array_equal(slipped, brute_dequant(codes, c2, c1, N, K))

@@ -5,9 +5,9 @@ operators run inside a host framework that owns the device memory pool and
 forbids allocation while it executes them, or serving loops that must not
 call cudaMalloc after start-up.  Instead of a caller workspace it uses a
 static 8 MiB device array inside the library.  Checked here through the C ABI
-against the regular forward (with a caller workspace), within the parity
-tolerance, on two calls in a row (the array keeps the previous call's
-contents), and for its size limit.  This file sorts last so a run that stops
+against the regular forward (with a caller workspace), bit for bit, on two
+calls in a row, each right after a call on another problem (the array keeps
+the previous call's contents), and for its size limit.  This file sorts last so a run that stops
 at the first failure has run everything else before it.
 """
 
@@ -39,25 +39,40 @@ def _noalloc(q, X, w, L1, L2, s, Y, T, status):
                                             ctypes.c_void_p(status.data_ptr()), stream)
 
 
-@pytest.mark.parametrize("M,N,K,r", [(16, 4096, 4096, 16), (200, 384, 512, 64), (37, 136, 256, 32)])
-def test_noalloc_forward_matches_regular_forward(lib, M, N, K, r):
-    rng = np.random.default_rng(M + N + K + r)
+def _problem(lib, rng, M, N, K, r):
     X, W = _bf(rng, (M, K), 1.0), _bf(rng, (N, K), 0.02)
     L1, L2 = _bf(rng, (K, r), K ** -0.5), _bf(rng, (r, N), 0.05)
-    s = 16.0 / r
+    return X, lib.quantize(W), L1, L2, 16.0 / r
+
+
+@pytest.mark.parametrize("M,N,K,r", [(16, 4096, 4096, 16), (200, 384, 512, 64), (37, 136, 256, 32),
+                                     (5, 2056, 1536, 8)])
+def test_noalloc_forward_matches_regular_forward(lib, M, N, K, r):
+    """Bit for bit the regular forward's result (the same kernels and launch
+    plan), on two calls in a row, each after the array was left holding
+    another problem's workspace: a different token regime (few-token GEMV
+    path against the tcgen05 engine), rank and data."""
+    rng = np.random.default_rng(M + N + K + r)
+    X, w, L1, L2, s = _problem(lib, rng, M, N, K, r)
     assert lib.workspace_bytes(M, N, K, r) <= 8 << 20
-    w = lib.quantize(W)
     Y_ref, T_ref = lib.linear_fwd(X, w, L1, L2, s)
+    # the other problem: few tokens if this one has many, and the reverse
+    pM, pr = (300, 48) if M <= 16 else (9, 128)
+    pX, pw, pL1, pL2, ps = _problem(lib, np.random.default_rng(7), pM, 1024, 512, pr)
+    pY = torch.empty((pM, 1024), dtype=torch.bfloat16, device="cuda")
+    pT = torch.empty((pM, pr), dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     for _ in range(2):
+        assert _noalloc(lib, pX, pw, pL1, pL2, ps, pY, pT, status) == 0
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         T = torch.full((M, r), float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc(lib, X, w, L1, L2, s, Y, T, status) == 0
         torch.cuda.synchronize()
         assert int(status.item()) == 0
+        assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16)), "Y differs from the regular forward"
+        assert torch.equal(T.view(torch.int32), T_ref.view(torch.int32)), "T differs from the regular forward"
         assert_close(to_f64(Y), to_f64(Y_ref), "Y")
-        assert_close(to_f64(T), to_f64(T_ref), "T")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
