@@ -17,6 +17,10 @@ Sources (the pages the method is taken from):
     BFloat16 for the matrix multiply).
   * tecyfy "What is QLoRA", section "The 3 tricks"; examadda "QLoRA",
     sections "The Core Idea" and "The Three Innovations".
+  * examadda "QLoRA", "Practical Notes" (merging an adapter into a 4-bit
+    base is lossy: dequantise first) and the paged-optimizer passages
+    (``adapters.py``).
 """
 
 from .nf4_oracle import *  # noqa: F401,F403
+from .adapters import *  # noqa: F401,F403
