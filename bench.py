@@ -28,7 +28,8 @@ At N = 1 it adds the other workloads as extra keys: llama7b_block (the same
 step on a LLaMA-7B block), linear4096_m16 (one 4096x4096 linear at 16
 tokens, fwd + bwd, against its HBM roofline), gemv (few-token forward of
 the LLaMA-65B FFN linears), quant / dequant / formats (the bulk 2^31-weight
-round trip) and context_bf16_gemm (cuBLAS on the dequantised weight).
+round trip), adapters (adapter merge and the paged AdamW step) and
+context_bf16_gemm (cuBLAS on the dequantised weight).
 `--impl reference` times the oracle as the reference arm.
 """
 
@@ -464,6 +465,58 @@ def few_token_linear(q, WL, dev, hbm_gbs, pk_kind, reps=50):
             "flops": linear_flops(M, N, K, r)}
 
 
+def adapter_rates(q, WL, dev, hbm_gbs, pk_kind, reps=10):
+    """Adapter merge of the LLaMA-65B gate linear (22016x8192, r = 64) and
+    the paged AdamW step over all adapters of the LLaMA-65B block (state in
+    paged memory, resident on the GPU), as GB/s of their algorithmic bytes
+    against the HBM copy bandwidth."""
+    import torch
+    wl = WL.WORKLOADS["llama65b_block"]
+    lin = wl.linears[4]
+    t = WL.make_linear(wl, lin, seed=4, device=dev, M=1)
+    w = q.quantize(t["W"])
+    del t["W"]
+    out = torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev)
+    for _ in range(2):
+        q.adapter_merge(w, t["L1"], t["L2"], wl.s, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        q.adapter_merge(w, t["L1"], t["L2"], wl.s, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    m_us = e0.elapsed_time(e1) * 1e3 / reps
+    m_bytes = nf4_bytes(lin.N, lin.K) + 2 * lin.N * lin.K + 2 * wl.r * (lin.N + lin.K)
+    del w, out, t
+    n = sum(wl.r * (l.N + l.K) for l in wl.linears)
+    p = torch.randn(n, device=dev) * 0.01
+    g = torch.randn(n, device=dev) * 1e-3
+    pb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    mb, vb = q.paged_empty(n, dev), q.paged_empty(n, dev)
+    mb.prefetch(dev.index or 0)
+    vb.prefetch(dev.index or 0)
+    for k in range(1, 3):
+        q.adamw_step(p, g, mb.tensor, vb.tensor, k, lr=1e-4, weight_decay=0.01, p_bf16=pb)
+    torch.cuda.synchronize()
+    e0.record()
+    for k in range(3, 3 + reps):
+        q.adamw_step(p, g, mb.tensor, vb.tensor, k, lr=1e-4, weight_decay=0.01, p_bf16=pb)
+    e1.record()
+    torch.cuda.synchronize()
+    a_us = e0.elapsed_time(e1) * 1e3 / reps
+    a_bytes = n * (4 * 2 + 4 + 4 * 2 + 4 * 2 + 2)   # p r/w, g, m r/w, v r/w, bf16 copy
+    assert q.read_status(dev) == 0
+    del mb, vb
+    return {
+        "merge": {"workload": f"W^ + s (L1 L2)^T of {lin.name} {lin.N}x{lin.K}, r={wl.r}, to bf16", "us": m_us,
+                  "bytes": m_bytes, "gbs": m_bytes / m_us / 1e3, "frac": m_bytes / m_us / 1e3 / hbm_gbs},
+        "adamw_paged": {"workload": f"AdamW over the {n} adapter parameters of the LLaMA-65B block (r={wl.r}), "
+                                    "state in paged memory resident on the GPU", "us": a_us, "bytes": a_bytes,
+                        "gbs": a_bytes / a_us / 1e3, "frac": a_bytes / a_us / 1e3 / hbm_gbs},
+        "peak": hbm_gbs, "peak_source": f"{pk_kind} HBM copy"}
+
+
 def bf16_gemm_ms(layers, reps):
     """Mean device time per step of the two weight products of every linear,
     Y = X.W^T and dX = dY.W, done by torch.matmul (cuBLAS) on the dequantised
@@ -657,6 +710,8 @@ def run_ours(args):
         line_extra["formats"] = {"workload": RT_WORKLOAD + "; FP4 = E2M1/6 and Int4 = k/7 levels (the compared "
                                                            "formats), nf4_e5m2 = NF4 with E5M2 block scales",
                                  "unit": "GB/s", **formats}
+        # ---- adapter merge and the paged AdamW step
+        line_extra["adapters"] = adapter_rates(q, WL, dev, hbm, pk_kind)
         # ---- few-token forward (dequant-GEMV regime): LLaMA-65B FFN up and down
         if not args.no_gemv:
             line_extra["gemv"] = gemv_rates(q, WL, dev, hbm, pk_kind)

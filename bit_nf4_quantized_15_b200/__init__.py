@@ -24,6 +24,7 @@ __all__ = [
     "lib", "NF4Weight", "quantize", "quantize_into", "dequant", "workspace_bytes", "linear_fwd", "linear_bwd",
     "codebook", "FORMATS", "SCALES", "status_string", "kernel_launches", "set_gemm_events",
     "debug_stall_next_gemm", "read_status", "storage_bytes", "LIB_PATH", "QLoRAError",
+    "adapter_merge", "adamw_step", "PagedBuffer", "paged_empty",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
@@ -50,6 +51,11 @@ class qlora_nf4_weight(ctypes.Structure):
                 ("format", ctypes.c_int32), ("scale_codec", ctypes.c_int32)]
 
 
+class qlora_adamw_config(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double), ("step", ctypes.c_int64)]
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -70,6 +76,12 @@ _SIGS = {
     "qlora_kernel_launches": (ctypes.c_uint64, []),
     "qlora_set_gemm_events": (ctypes.c_int, [_P, _P]),
     "qlora_debug_stall_next_gemm": (ctypes.c_int, [ctypes.c_uint64]),
+    "qlora_adapter_merge": (ctypes.c_int, [ctypes.POINTER(qlora_nf4_weight), _P, _P, ctypes.c_int, ctypes.c_float,
+                                           _P, _P, _P]),
+    "qlora_adamw_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, ctypes.c_void_p, _P]),
+    "qlora_paged_alloc": (ctypes.c_int, [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]),
+    "qlora_paged_free": (ctypes.c_int, [_P]),
+    "qlora_paged_prefetch": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_int, _P]),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P, ctypes.c_int,
                                                 ctypes.c_float, _P, _P, _P, _P]),
 }
@@ -280,3 +292,66 @@ def linear_bwd(dY, X, T, w: NF4Weight, L1, L2, s: float, ws=None, need_dX=True, 
                                   _ptr(dX), _ptr(dL1), _ptr(dL2), _ptr(ws), ws.numel(),
                                   _ptr(status if status is not None else _status(dev)), _stream(dev)))
     return dX, dL1, dL2
+
+
+def adapter_merge(w: NF4Weight, L1, L2, s: float, out=None, status=None) -> torch.Tensor:
+    """W_merged = RNbf16(W^ + s (L1 L2)^T) as a bf16 [N, K] tensor (the adapter
+    folded into the dequantised weight; quantize() it again for a 4-bit copy)."""
+    _bf16_cuda(L1, "L1"), _bf16_cuda(L2, "L2")
+    r = L1.shape[1]
+    dev = w.device
+    if out is None:
+        out = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=dev)
+    d = w.descriptor()
+    _check(lib().qlora_adapter_merge(ctypes.byref(d), _ptr(L1), _ptr(L2), r, float(s), _ptr(out),
+                                     _ptr(status if status is not None else _status(dev)), _stream(dev)))
+    return out
+
+
+def adamw_step(p, g, m, v, step: int, lr: float, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
+               p_bf16=None):
+    """One AdamW step in place on fp32 p, m, v (device or paged memory) for
+    the gradient g; writes RNbf16(p) into p_bf16 when given."""
+    for t, name in ((p, "p"), (g, "g"), (m, "m"), (v, "v")):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != p.numel():
+            raise QLoRAError(f"{name} must be a contiguous float32 tensor of p's size")
+    if p_bf16 is not None and (p_bf16.dtype != torch.bfloat16 or p_bf16.numel() != p.numel()):
+        raise QLoRAError("p_bf16 must be a bf16 tensor of p's size")
+    cfg = qlora_adamw_config(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
+    _check(lib().qlora_adamw_step(_ptr(p), _ptr(p_bf16), _ptr(g), _ptr(m), _ptr(v), p.numel(),
+                                  ctypes.cast(ctypes.byref(cfg), ctypes.c_void_p), _stream(p.device)))
+
+
+class PagedBuffer:
+    """fp32 optimizer state in paged (CUDA managed) memory from
+    qlora_paged_alloc; ``tensor`` views it as a CUDA tensor without a copy.
+    ``prefetch(device)`` moves it ahead of use (-1: host memory)."""
+
+    def __init__(self, n: int, device="cuda"):
+        self.n = int(n)
+        self.device = torch.device(device)
+        ptr = ctypes.c_void_p()
+        _check(lib().qlora_paged_alloc(max(self.n, 1) * 4, ctypes.byref(ptr)))
+        self.ptr = ptr.value
+        self.__cuda_array_interface__ = {"shape": (self.n,), "typestr": "<f4", "data": (self.ptr, False),
+                                         "version": 3, "strides": None}
+        self.tensor = torch.as_tensor(self, device=self.device)
+
+    def prefetch(self, device: int, stream=None):
+        st = ctypes.c_void_p(torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream)
+        _check(lib().qlora_paged_prefetch(ctypes.c_void_p(self.ptr), self.n * 4, int(device), st))
+
+    def __del__(self):
+        try:
+            if getattr(self, "ptr", None) and _lib is not None:
+                _lib.qlora_paged_free(ctypes.c_void_p(self.ptr))
+                self.ptr = None
+        except Exception:
+            pass
+
+
+def paged_empty(n: int, device="cuda") -> "PagedBuffer":
+    """A zeroed fp32 paged buffer of n elements (optimizer state: m or v)."""
+    b = PagedBuffer(n, device)
+    b.tensor.zero_()
+    return b

@@ -3,6 +3,7 @@
 // synchronisation: all work is queued on the caller's stream.
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -402,6 +403,64 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
     if (int rc = run_timed(a, pair ? A_PAIR_K : A_DEQ_K, p, partial, st)) return rc;
   }
   return QLORA_OK;
+}
+
+int qlora_adapter_merge(const qlora_nf4_weight* w, const uint16_t* L1, const uint16_t* L2, int r, float s,
+                        uint16_t* W_out, int* status_dev, qlora_stream_t stream) {
+  (void)status_dev;
+  if (!w || !w->codes || !w->c2 || !w->c1 || !L1 || !L2 || !W_out) return QLORA_ERR_NULL;
+  const int64_t N = w->n_rows, K = w->n_cols;
+  if (!shape_ok(1, N, K)) return QLORA_ERR_SHAPE;
+  if (!format_ok(w)) return QLORA_ERR_FORMAT;
+  if (!valid_rank(r)) return QLORA_ERR_RANK;
+  for (const void* p : {(const void*)w->codes, (const void*)L1, (const void*)L2, (const void*)W_out})
+    if (!aligned16(p)) return QLORA_ERR_ALIGN;
+  DevInfo di;
+  if (int rc = current_device_info(&di)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch_adapter_merge(w->codes, w->c2, w->c1, w->format, w->scale_codec, N, K, L1, L2, r, s, W_out, st) ==
+                 cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+int qlora_adamw_step(float* p, uint16_t* p_bf16, const float* g, float* m, float* v, int64_t n,
+                     const qlora_adamw_config* cfg, qlora_stream_t stream) {
+  if (!p || !g || !m || !v || !cfg) return QLORA_ERR_NULL;
+  if (n < 0 || cfg->step < 1) return QLORA_ERR_SHAPE;
+  for (const void* q : {(const void*)p, (const void*)g, (const void*)m, (const void*)v})
+    if (!aligned16(q)) return QLORA_ERR_ALIGN;
+  if (p_bf16 && (reinterpret_cast<uintptr_t>(p_bf16) & 7u)) return QLORA_ERR_ALIGN;
+  if (n == 0) return QLORA_OK;
+  DevInfo di;
+  if (int rc = current_device_info(&di)) return rc;
+  // every constant computed in double and rounded once to float
+  const double t = (double)cfg->step;
+  const float sc[9] = {(float)cfg->lr, (float)cfg->beta1, (float)(1.0 - cfg->beta1), (float)cfg->beta2,
+                       (float)(1.0 - cfg->beta2), (float)cfg->eps, (float)cfg->weight_decay,
+                       (float)(1.0 - std::pow(cfg->beta1, t)), (float)(1.0 - std::pow(cfg->beta2, t))};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch_adamw(p, p_bf16, g, m, v, n, sc, st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+int qlora_paged_alloc(size_t bytes, void** out) {
+  if (!out) return QLORA_ERR_NULL;
+  *out = nullptr;
+  if (bytes == 0) return QLORA_ERR_SHAPE;
+  return cudaMallocManaged(out, bytes, cudaMemAttachGlobal) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+int qlora_paged_free(void* p) {
+  if (!p) return QLORA_OK;
+  return cudaFree(p) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+int qlora_paged_prefetch(const void* p, size_t bytes, int device, qlora_stream_t stream) {
+  if (!p) return QLORA_ERR_NULL;
+  if (bytes == 0) return QLORA_OK;
+  const int dst = device < 0 ? cudaCpuDeviceId : device;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return cudaMemPrefetchAsync(p, bytes, dst, st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const float* T_saved,

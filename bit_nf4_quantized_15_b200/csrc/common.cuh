@@ -83,6 +83,26 @@ QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, in
   }
 }
 
+// The same bounded wait for a thread that is not on the critical path (a
+// producer refilling a ring that is usually full): it sleeps between polls
+// so that its spinning does not take issue slots from the warps that work.
+QDEV bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                            uint32_t sleep_ns, uint64_t limit_ns = QNF4_WAIT_NS) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      report(status, QLORA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Short bounded wait used only while draining after an abort.
 QDEV void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t ns) {
   const uint32_t a = smem_u32(bar);

@@ -30,15 +30,17 @@
 //   its rows, i.e. k = 16c .. 16c+15, handing k-step s the pairs 2s (A
 //   columns 2c, 2c+1) and 2s+1 (columns 2c+8, 2c+9), and reads the matching
 //   X values k = 16c+4s .. 16c+4s+3 as one 8-byte load.
-//   Dequantisation uses a 64 KB shared-memory table of code pairs: entry e
+//   The block scale is applied after the product: a weight row's 64-wide
+//   block contributes c^ . sum_k x[k] q[code_k] (one fp32 multiply-add per
+//   accumulator element after the block's four MMAs, which start from zero),
+//   the same sum as sum_k x[k] (q[code_k] c^) up to rounding, within the
+//   layer's stated tolerance.  So the A operand is the level itself, and a
+//   32 KB shared-memory table of code pairs serves the whole kernel: entry e
 //   (one code byte: element 2j in the low nibble, 2j+1 in the high one) holds
-//   the fp32 levels (q[e & 15], q[e >> 4]), replicated for the 32 lanes so a
-//   warp's 8-byte loads never collide in a bank.  Per code byte: one byte
-//   permute forms the address, one LDS.64 fetches both levels, one packed
-//   multiply by the block scale c^ gives RN32(q.c^) for both weights and one
-//   conversion rounds the pair to bf16, i.e. exactly
-//   RNbf16(RN32(q[code].c^)), the dequantised weight of the pages; that
-//   bf16 pair is one A-fragment register.
+//   the bf16 pair (RNbf16(q[e & 15]), RNbf16(q[e >> 4])), one copy per lane at
+//   a 4-byte offset so a warp's loads fall in 32 different banks.  Per code
+//   byte: one byte permute forms the address and one 4-byte load fetches the
+//   A-fragment register for both weights.
 //   Warp 0: lanes 0..2 are the three TMA producers; the last warp sums this
 //   CTA's share of the T partials.
 // * gemv_finish_kernel: per row, the row tile's segment partials in worker
@@ -62,7 +64,7 @@ constexpr int kWW = 8 / kRG;                  // warps per worker
 // Warps: 0 producers, 1 .. kWW*kWG workers, last: T reduction.
 constexpr int kWarpT = 1 + kWW * kWG;
 constexpr int kGThreads = 32 * (kWarpT + 1);
-constexpr int kTabBytes = 65536;           // 256 pairs x 32 lanes x 8 bytes
+constexpr int kTabBytes = 65536;           // 256 pairs x 256-byte lines (32 lanes x 4 bytes used)
 constexpr int kBarBytes = 1024;
 // Shared window: two stages and the barriers, then (at the next 64 KB
 // boundary, so the table's address bits 16.. come from one register in the
@@ -115,24 +117,20 @@ __host__ __device__ __forceinline__ int worker_of(int64_t u, int64_t U, int W) {
   return (int)(((u + 1) * (int64_t)W - 1) / U);
 }
 
-QDEV float2 lds_pair(uint32_t addr) {
-  float2 v;
-  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
 QDEV uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 
-// bf16x2 of code byte k (0..3) of word w: RNbf16(RN32(q[lo].c^)) low half,
-// RNbf16(RN32(q[hi].c^)) high half.  lanereg = table address bits 16..23 in
-// byte 2, lane * 8 in byte 0.
-QDEV uint32_t pair_lookup(uint32_t w, int k, uint32_t lanereg, float2 cc) {
+// bf16x2 of code byte k (0..3) of word w: RNbf16(q[lo]) low half,
+// RNbf16(q[hi]) high half.  lanereg = table address bits 16..23 in byte 2,
+// lane * 4 in byte 0; the code byte becomes address byte 1.
+QDEV uint32_t pair_lookup(uint32_t w, int k, uint32_t lanereg) {
   const uint32_t addr = __byte_perm(w, lanereg, 0x7604u | ((uint32_t)k << 4));
-  const float2 p = __fmul2_rn(lds_pair(addr), cc);
-  return pack_bf16x2(p.x, p.y);
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 QDEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -176,10 +174,28 @@ QDEV RowScales load_row_scales(const GemvArgs& a, int rt, int un, int rl) {
   s.c1b = __ldg(a.c1 + ((f0 + nkb - 1) >> 8));
   return s;
 }
-// c^ of k block q (0..3) of the unit whose first block is f0's.
-QDEV float row_chat(const RowScales& s, int q, int64_t f0, bool e5m2) {
-  const float c1 = ((f0 + q) >> 8) == (f0 >> 8) ? s.c1a : s.c1b;
-  return decode_scale((s.c2 >> (8 * q)) & 0xFFu, c1, e5m2);
+// c^ = RN32(dec(c2) . c1) of the unit's four k blocks for one row, whose
+// first block has flat index f0 (block q lies in the next c1 group when
+// (f0 mod 256) + q >= 256).  Two codes per conversion: an E4M3 pair through
+// the hardware fp8x2 -> f16x2 conversion, an E5M2 byte as the high byte of
+// an fp16; both exact.
+QDEV void row_chats(const RowScales& s, int64_t f0, bool e5m2, float (&out)[kUnitKB]) {
+  float2 v01, v23;
+  if (e5m2) {
+    const uint32_t b01 = __byte_perm(s.c2, 0u, 0x1404u), b23 = __byte_perm(s.c2, 0u, 0x3424u);
+    v01 = __half22float2(*reinterpret_cast<const __half2*>(&b01));
+    v23 = __half22float2(*reinterpret_cast<const __half2*>(&b23));
+  } else {
+    const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(s.c2 & 0xFFFFu), __NV_E4M3);
+    const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(s.c2 >> 16), __NV_E4M3);
+    v01 = __half22float2(__half2(h01));
+    v23 = __half22float2(__half2(h23));
+  }
+  const int g0 = (int)(f0 & 255);
+  out[0] = __fmul_rn(v01.x, g0 + 0 < 256 ? s.c1a : s.c1b);
+  out[1] = __fmul_rn(v01.y, g0 + 1 < 256 ? s.c1a : s.c1b);
+  out[2] = __fmul_rn(v23.x, g0 + 2 < 256 ? s.c1a : s.c1b);
+  out[3] = __fmul_rn(v23.y, g0 + 3 < 256 ? s.c1a : s.c1b);
 }
 
 // NT = 8-token column tiles (1 for M <= 8, 2 for M <= 16).
@@ -210,12 +226,11 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
     tma_prefetch_desc(&args.tmCodes);
     tma_prefetch_desc(&args.tmX);
   }
-  // Pair table: entry e, lane l at tab + e*256 + l*8.
+  // Pair table: entry e, lane l at tab + e*256 + l*4.
   for (int idx = tid; idx < 256 * 32; idx += kGThreads) {
     const int e = idx >> 5, l = idx & 31;
-    const float lo = args.q[e & 15], hi = args.q[e >> 4];
-    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(S.tab + (uint32_t)(e * 256 + l * 8)), "f"(lo), "f"(hi)
-                 : "memory");
+    const uint32_t v = pack_bf16x2(args.q[e & 15], args.q[e >> 4]);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(S.tab + (uint32_t)(e * 256 + l * 4)), "r"(v) : "memory");
   }
   __syncthreads();
 
@@ -228,7 +243,8 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
       int issued = 0;
       for (int i = 0; i < nu; ++i) {
         const int j = i % kWS;
-        if (!mbar_wait(bar_empty(S, g, j), ((uint32_t)(i / kWS) & 1u) ^ 1u, S.abort_flag, args.status)) break;
+        if (!mbar_wait_backoff(bar_empty(S, g, j), ((uint32_t)(i / kWS) & 1u) ^ 1u, S.abort_flag, args.status, 128))
+          break;
         const int64_t u = u0 + i;
         const int rt = (int)(u / upr), un = (int)(u % upr);
         const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);  // k blocks of W in this unit
@@ -276,7 +292,7 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
     int rows[2 * kRG];
 #pragma unroll
     for (int i = 0; i < 2 * kRG; ++i) rows[i] = wq * 16 * kRG + (i >> 1) * 16 + (i & 1) * 8 + gr;
-    const uint32_t lanereg = (S.tab & 0x00FF0000u) | (uint32_t)(lane * 8);
+    const uint32_t lanereg = (S.tab & 0x00FF0000u) | (uint32_t)(lane * 4);
     const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
     const int nu = (int)(u1 - u0);
     float acc[kRG][NT][4];
@@ -297,9 +313,10 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
       const int rt = (int)(u / upr), un = (int)(u % upr);
       const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);
       const bool seg_end = i == nu - 1 || un == upr - 1;
-      RowScales cur[2 * kRG];
+      float chs[2 * kRG][kUnitKB];  // c^ of this unit's blocks, per thread row
 #pragma unroll
-      for (int r = 0; r < 2 * kRG; ++r) cur[r] = sc[r];
+      for (int r = 0; r < 2 * kRG; ++r)
+        row_chats(sc[r], ((int64_t)rt * 128 + rows[r]) * args.kbt + (int64_t)un * kUnitKB, args.c2_e5m2 != 0, chs[r]);
       if (i + 1 < nu) {
 #pragma unroll
         for (int r = 0; r < 2 * kRG; ++r) sc[r] = load_row_scales(args, (int)((u + 1) / upr), (int)((u + 1) % upr), rows[r]);
@@ -326,29 +343,37 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
 #pragma unroll
           for (int h = 0; h < kRG; ++h) {  // 16-row group h: rows[2h] (gr) and rows[2h+1] (gr + 8)
             uint2 cw[2];
-            float2 cc[2];
+            float ch[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int rl = rows[2 * h + e];
               cw[e] = lds64(st + (uint32_t)rl * 128 +
                             ((((uint32_t)(2 * q + (cq >> 1))) ^ (uint32_t)(rl & 7)) << 4) + 8u * (uint32_t)(cq & 1));
-              const int64_t f0 = ((int64_t)rt * 128 + rl) * args.kbt + (int64_t)un * kUnitKB;
-              const float ch = row_chat(cur[2 * h + e], q, f0, args.c2_e5m2 != 0);
-              cc[e] = make_float2(ch, ch);
+              ch[e] = chs[2 * h + e][q];
             }
+            float blk[NT][4];
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) blk[t][e] = 0.0f;
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
               // code bytes 2s and 2s+1 of the thread's 8: word s >> 1, bytes 2(s&1), 2(s&1)+1
               const uint32_t w0 = (s < 2) ? cw[0].x : cw[0].y;
               const uint32_t w1 = (s < 2) ? cw[1].x : cw[1].y;
               const int k0 = 2 * (s & 1);
-              const uint32_t a0 = pair_lookup(w0, k0, lanereg, cc[0]);
-              const uint32_t a1 = pair_lookup(w1, k0, lanereg, cc[1]);
-              const uint32_t a2 = pair_lookup(w0, k0 + 1, lanereg, cc[0]);
-              const uint32_t a3 = pair_lookup(w1, k0 + 1, lanereg, cc[1]);
+              const uint32_t a0 = pair_lookup(w0, k0, lanereg);
+              const uint32_t a1 = pair_lookup(w1, k0, lanereg);
+              const uint32_t a2 = pair_lookup(w0, k0 + 1, lanereg);
+              const uint32_t a3 = pair_lookup(w1, k0 + 1, lanereg);
 #pragma unroll
-              for (int t = 0; t < NT; ++t) mma_bf16_16816(acc[h][t], a0, a1, a2, a3, xb[t][s].x, xb[t][s].y);
+              for (int t = 0; t < NT; ++t) mma_bf16_16816(blk[t], a0, a1, a2, a3, xb[t][s].x, xb[t][s].y);
             }
+            // the block's scale: accumulator elements 0, 1 are row gr, 2, 3 row gr + 8
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[h][t][e] = __fmaf_rn(blk[t][e], ch[e >> 1], acc[h][t][e]);
           }
         }
       }

@@ -161,4 +161,14 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* c2, const float*
                            uint16_t* out, int format, int scale_codec, cudaStream_t st);
 cudaError_t launch_scale_to_bf16(const float* in, int64_t n, float s, uint16_t* out, cudaStream_t st);
 
+// ------------------------------------------------------- adapter kernels
+// W_merged = RNbf16(W^ + s (L1 L2)^T), one CTA per 128 x 128 output tile.
+size_t merge_smem_bytes(int r);
+cudaError_t launch_adapter_merge(const uint8_t* codes, const uint8_t* c2, const float* c1, int format, int scale_codec,
+                                 int64_t N, int64_t K, const uint16_t* L1, const uint16_t* L2, int r, float s,
+                                 uint16_t* out, cudaStream_t st);
+// AdamW step; sc = lr, b1, 1-b1, b2, 1-b2, eps, wd, 1-b1^t, 1-b2^t (fp32).
+cudaError_t launch_adamw(float* p, uint16_t* pb, const float* g, float* m, float* v, int64_t n, const float* sc,
+                         cudaStream_t st);
+
 }  // namespace qnf4

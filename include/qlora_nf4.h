@@ -14,8 +14,10 @@
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers, owned and allocated by the
- *     caller.  The library never allocates, frees or synchronises; every call
- *     is asynchronous on `stream` (a cudaStream_t, 0 = legacy default).
+ *     caller.  The library never allocates, frees or synchronises (except
+ *     the paged-state helpers qlora_paged_alloc / qlora_paged_free, whose job
+ *     is to allocate); every call is asynchronous on `stream` (a
+ *     cudaStream_t, 0 = legacy default).
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - Tensors are dense row-major.  Every pointer must be 16-byte aligned.
  *   - Return value: QLORA_OK, or a negative QLORA_ERR_* from the host-side
@@ -195,6 +197,52 @@ QLORA_API int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M,
                      const qlora_nf4_weight* w, const uint16_t* L1, const uint16_t* L2, int r,
                      float s, uint16_t* dX, float* dL1, float* dL2, void* ws, size_t ws_bytes,
                      int* status_dev, qlora_stream_t stream);
+
+/*
+ * Adapter merge (examadda "QLoRA", "Practical Notes", third bullet: merging
+ * an adapter back into a 4-bit base is lossy, so dequantise first):
+ *   W_out = RNbf16( W^ + s . (L1 . L2)^T ),   W^ = doubleDequant(c1, c2, W_NF4)
+ * computed as RN32(W^ + s . acc) with acc the rank-r product accumulated in
+ * fp32 on the tensor cores (summation order unspecified), then rounded once
+ * to bf16.  W_out: device bf16[N][K] (the nn.Linear layout of W).  L1, L2 as
+ * in qlora_linear_fwd; same rank rules.  Quantising W_out again
+ * (qlora_nf4_quantize) is a separate, lossy step.
+ */
+QLORA_API int qlora_adapter_merge(const qlora_nf4_weight* w, const uint16_t* L1, const uint16_t* L2, int r,
+                                  float s, uint16_t* W_out, int* status_dev, qlora_stream_t stream);
+
+/*
+ * One AdamW step on the adapters (the optimizer whose state the paged
+ * optimizers keep in memory that moves between GPU and host: nlp-lineage
+ * "QLoRA", section "The idea", paged-optimizers bullet; inferensys glossary,
+ * paged-optimizers paragraph).  Decoupled weight decay, each operation
+ * rounded to fp32 in this order (t = step, constants computed in double and
+ * rounded once to float):
+ *   m = b1 m + (1 - b1) g;   v = b2 v + ((1 - b2) g) g
+ *   p = p - lr ( (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps) + wd p )
+ * p, g, m, v: float[n], 16-byte aligned, device or managed memory (see
+ * qlora_paged_alloc); p_bf16 (optional, 8-byte aligned) receives RNbf16(p),
+ * the copy the layer multiplies with.  Updates p, m, v in place.
+ */
+typedef struct qlora_adamw_config {
+  double lr, beta1, beta2, eps, weight_decay;
+  int64_t step; /* 1 for the first step */
+} qlora_adamw_config;
+
+QLORA_API int qlora_adamw_step(float* p, uint16_t* p_bf16, const float* g, float* m, float* v, int64_t n,
+                               const qlora_adamw_config* cfg, qlora_stream_t stream);
+
+/*
+ * Paged optimizer state: memory that the driver pages between the GPU and
+ * host memory on demand (CUDA managed memory), so optimizer state can exceed
+ * the GPU's free memory for a moment without failing.  These are the only
+ * calls of the library that allocate or free.  qlora_paged_prefetch moves a
+ * range ahead of use: device >= 0 to that GPU, -1 to host memory; it is
+ * asynchronous on `stream`.
+ */
+QLORA_API int qlora_paged_alloc(size_t bytes, void** out);
+QLORA_API int qlora_paged_free(void* p);
+QLORA_API int qlora_paged_prefetch(const void* p, size_t bytes, int device, qlora_stream_t stream);
 
 /*
  * Forward without a caller workspace, for callers that cannot allocate

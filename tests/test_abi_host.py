@@ -126,3 +126,28 @@ def test_format_checks_before_any_launch(q):
         assert L.qlora_linear_bwd(fake, fake, 4, fake, ctypes.byref(w), fake, fake, 16, 1.0, fake, None, None,
                                   fake, 1 << 20, None, None) == -11
     assert "format" in q.status_string(-11)
+
+
+def test_adapter_entry_points_check_arguments_before_any_launch(q):
+    """Merge and AdamW reject bad arguments on the host (fake pointers that
+    would fault if a kernel ran); the paged helpers reject NULL."""
+    L = q.lib()
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    w = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 128)
+    assert L.qlora_adapter_merge(ctypes.byref(w), None, fake, 16, 1.0, fake, None, None) == -1
+    assert L.qlora_adapter_merge(ctypes.byref(w), fake, fake, 12, 1.0, fake, None, None) == -4
+    assert L.qlora_adapter_merge(ctypes.byref(w), fake, fake, 16, 1.0, P(0x10002), None, None) == -2
+    w_bad = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 96)
+    assert L.qlora_adapter_merge(ctypes.byref(w_bad), fake, fake, 16, 1.0, fake, None, None) == -3
+    cfg = q.qlora_adamw_config(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    pc = ctypes.cast(ctypes.byref(cfg), ctypes.c_void_p)
+    assert L.qlora_adamw_step(fake, None, fake, fake, P(0x10004), 100, pc, None) == -2
+    assert L.qlora_adamw_step(fake, P(0x20002), fake, fake, fake, 100, pc, None) == -2
+    assert L.qlora_adamw_step(fake, None, None, fake, fake, 100, pc, None) == -1
+    cfg0 = q.qlora_adamw_config(1e-3, 0.9, 0.999, 1e-8, 0.0, 0)
+    assert L.qlora_adamw_step(fake, None, fake, fake, fake, 100, ctypes.cast(ctypes.byref(cfg0), ctypes.c_void_p),
+                              None) == -3
+    assert L.qlora_adamw_step(fake, None, fake, fake, fake, 0, pc, None) == 0      # nothing to do
+    assert L.qlora_paged_alloc(16, None) == -1 and L.qlora_paged_prefetch(None, 16, 0, None) == -1
+    assert L.qlora_paged_free(None) == 0
