@@ -31,6 +31,7 @@ __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits", "bf16_bits_to_f64",
     "e4m3_decode", "e4m3_encode", "e4m3_encode_exact",
     "E5M2_MAX", "SCALE_CODECS", "e5m2_decode", "e5m2_encode", "e5m2_encode_exact",
+    "MEAN_CODECS", "pairwise_sum_f32",
     "block_absmax", "quantize", "dequant", "decoded_scales",
     "linear_fwd", "linear_bwd", "adapter_grads",
     "storage_bytes", "bits_per_weight",
@@ -362,7 +363,36 @@ def e5m2_encode(x: np.ndarray) -> np.ndarray:
 
 
 # scale codec -> (largest finite value, encoder, decoder)
-SCALE_CODECS = {"e4m3": (E4M3_MAX, e4m3_encode, e4m3_decode), "e5m2": (E5M2_MAX, e5m2_encode, e5m2_decode)}
+SCALE_CODECS = {"e4m3": (E4M3_MAX, e4m3_encode, e4m3_decode), "e5m2": (E5M2_MAX, e5m2_encode, e5m2_decode),
+                "e4m3_mean": (E4M3_MAX, e4m3_encode, e4m3_decode)}
+# Codecs whose c1 array holds two fp32 values per group: c1_g, then the group
+# mean mu_g of the block scales (the mean-centred double quantisation).
+MEAN_CODECS = ("e4m3_mean",)
+
+
+# ---------------------------------------------------------------------------
+# Mean-centred double quantisation (a variant of the scale quantisation; the
+# pages say only that the 32-bit block scales are quantised to 8-bit floats,
+# inferensys glossary, double-quantisation paragraph).  Reading: all block
+# scales are non-negative, so before the 8-bit step each group of 256 is
+# centred on its mean and the signed residuals use the sign bit of E4M3:
+#   mu_g = RN32(S_g / n_g), S_g the fp32 sum of the group's scales taken as a
+#          pairwise tree over 256 slots (adjacent pairs first, empty slots of
+#          a partial group are zeros), n_g the number of blocks in the group
+#   d_b  = RN32(c_b - mu_g);  c1_g = RN32(max_b |d_b| / 448)
+#   c2_b = E4M3_RNE_sat(RN32(d_b / c1_g)), signed; 0 when c1_g = 0
+#   c^_b = RN32(RN32(dec(c2_b) * c1_g) + mu_g)
+# ---------------------------------------------------------------------------
+
+def pairwise_sum_f32(v: np.ndarray, slots: int = DQ_BLOCK) -> np.float32:
+    """fp32 sum of ``v`` (at most ``slots`` values, zero-padded) as a pairwise
+    tree: slot 2i + slot 2i+1 first, then pairs of those sums, ... ; every
+    addition rounded to fp32."""
+    a = np.zeros(slots, np.float32)
+    a[: len(v)] = np.asarray(v, np.float32)
+    while len(a) > 1:
+        a = (a[0::2] + a[1::2]).astype(np.float32)
+    return np.float32(a[0])
 
 
 # ---------------------------------------------------------------------------
@@ -384,7 +414,9 @@ def _check_shape(N: int, K: int):
 def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16, fmt: str = "nf4", scale: str = "e4m3"):
     """NF4 double quantisation of a bf16 weight ``[N, K]`` (``fmt`` swaps the
     16 levels for one of the compared formats, see :func:`codebook`;
-    ``scale="e5m2"`` stores c2 as E5M2 with c1 = RN32(max / 57344)).
+    ``scale="e5m2"`` stores c2 as E5M2 with c1 = RN32(max / 57344);
+    ``scale="e4m3_mean"`` centres each group on its mean first, see
+    :data:`MEAN_CODECS`, and returns c1 as [c1_0, mu_0, c1_1, mu_1, ...]).
 
     Returns ``(codes, c2, c1)``:
       * ``codes`` uint8 ``[N*K/2]``: element 2j in the low nibble, 2j+1 in the
@@ -421,24 +453,37 @@ def quantize(W_bits: np.ndarray, chunk_blocks: int = 1 << 16, fmt: str = "nf4", 
         code = nearest_level(x, q)
         codes[b0:b0 + chunk_blocks] = code[:, 0::2] | (code[:, 1::2] << 4)
     G = (nb + DQ_BLOCK - 1) // DQ_BLOCK
-    c1 = np.empty(G, dtype=np.float32)
+    mean = scale in MEAN_CODECS
+    c1 = np.empty(2 * G if mean else G, dtype=np.float32)
     c2 = np.empty(nb, dtype=np.uint8)
     smax, encode, _ = SCALE_CODECS[scale]
     for g in range(G):
         cg = absmax[g * DQ_BLOCK:(g + 1) * DQ_BLOCK]
-        c1g = np.float32(cg.max()) / np.float32(smax)       # fp32 division
-        c1[g] = c1g
+        if mean:
+            mu = np.float32(pairwise_sum_f32(cg) / np.float32(len(cg)))   # fp32 division
+            d = (cg - mu).astype(np.float32)                                # fp32 subtraction
+            c1g = np.float32(np.abs(d).max()) / np.float32(smax)
+            c1[2 * g], c1[2 * g + 1] = c1g, mu
+        else:
+            d = cg
+            c1g = np.float32(cg.max()) / np.float32(smax)       # fp32 division
+            c1[g] = c1g
         if c1g > 0:
-            c2[g * DQ_BLOCK:(g + 1) * DQ_BLOCK] = encode((cg / c1g).astype(np.float32))
+            c2[g * DQ_BLOCK:(g + 1) * DQ_BLOCK] = encode((d / c1g).astype(np.float32))
         else:
             c2[g * DQ_BLOCK:(g + 1) * DQ_BLOCK] = 0
     return codes.reshape(-1), c2, c1
 
 
 def decoded_scales(c2: np.ndarray, c1: np.ndarray, scale: str = "e4m3") -> np.ndarray:
-    """c^_b = RN32(dec(c2_b) * c1_g): the 32-bit scale used by the dequantiser."""
+    """c^_b = RN32(dec(c2_b) * c1_g): the 32-bit scale used by the dequantiser
+    (mean-centred codec: RN32(RN32(dec(c2_b) * c1_g) + mu_g), two fp32
+    operations, no fused multiply-add)."""
     dec = SCALE_CODECS[scale][2](c2).astype(np.float32)  # every 8-bit float value is exact in fp32
     g = np.arange(len(c2)) // DQ_BLOCK
+    if scale in MEAN_CODECS:
+        prod = (dec * c1[2 * g]).astype(np.float32)
+        return (prod + c1[2 * g + 1]).astype(np.float32)
     return (dec * c1[g]).astype(np.float32)             # fp32 multiply
 
 
@@ -515,12 +560,13 @@ def linear_bwd(dY, X, What, L1, L2, s, T=None):
 # scales to 8 bits).
 # ---------------------------------------------------------------------------
 
-def storage_bytes(N: int, K: int, double_quant: bool = True) -> int:
+def storage_bytes(N: int, K: int, double_quant: bool = True, scale: str = "e4m3") -> int:
     n = N * K
     nb = n // BLOCK
     if not double_quant:
         return n // 2 + 4 * nb
-    return n // 2 + nb + 4 * ((nb + DQ_BLOCK - 1) // DQ_BLOCK)
+    per_group = 8 if scale in MEAN_CODECS else 4
+    return n // 2 + nb + per_group * ((nb + DQ_BLOCK - 1) // DQ_BLOCK)
 
 
 def bits_per_weight(N: int, K: int, double_quant: bool = True) -> float:
