@@ -36,9 +36,10 @@ QLORA_ERR_TIMEOUT = -8
 # Code formats (QLORA_FMT_*): NF4, and the two 4-bit formats the method is
 # compared with (FP4 = E2M1/6, Int4 = k/7).
 FORMATS = {"nf4": 0, "fp4": 1, "int4": 2}
-# Codec of the 8-bit block scales c2 (QLORA_SCALE_*): E4M3, or E5M2 as the
-# compared alternative.
-SCALES = {"e4m3": 0, "e5m2": 1}
+# Codec of the 8-bit block scales c2 (QLORA_SCALE_*): E4M3, E5M2 as the
+# compared alternative, or E4M3 of the residuals from each group's mean
+# (mean-centred; c1 then holds [c1, mean] per group).
+SCALES = {"e4m3": 0, "e5m2": 1, "e4m3_mean": 2}
 
 
 class QLoRAError(RuntimeError):
@@ -63,6 +64,8 @@ _I64 = ctypes.c_int64
 _SIGS = {
     "qlora_nf4_storage_bytes": (ctypes.c_int, [_I64, _I64, ctypes.POINTER(ctypes.c_size_t),
                                                ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "qlora_weight_storage_bytes": (ctypes.c_int, [_I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t),
+                                                  ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
     "qlora_nf4_codebook": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float)]),
     "qlora_code_levels": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_float)]),
     "qlora_nf4_quantize": (ctypes.c_int, [_P, _I64, _I64, ctypes.POINTER(qlora_nf4_weight), _P, _P]),
@@ -169,15 +172,19 @@ def _bf16_cuda(t, name):
     return t
 
 
-def storage_bytes(N: int, K: int):
+def storage_bytes(N: int, K: int, scale: str = "e4m3"):
+    """(codes, c2, c1) bytes of an N x K weight with the given scale codec."""
+    if scale not in SCALES:
+        raise QLoRAError(f"unknown scale codec {scale!r}")
     a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
-    _check(lib().qlora_nf4_storage_bytes(N, K, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    _check(lib().qlora_weight_storage_bytes(N, K, SCALES[scale], ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
     return a.value, b.value, c.value
 
 
 @dataclass
 class NF4Weight:
-    """Quantized weight: codes uint8[N*K/2], c2 uint8[N*K/64] (E4M3), c1 float32[ceil(N*K/16384)];
+    """Quantized weight: codes uint8[N*K/2], c2 uint8[N*K/64] (E4M3), c1 float32[ceil(N*K/16384)]
+    (two per group for the mean-centred codec);
     ``fmt`` names the 16 levels the codes index (see FORMATS), ``scale`` the
     8-bit float of c2 (see SCALES)."""
     codes: torch.Tensor
@@ -200,7 +207,7 @@ class NF4Weight:
 
     @staticmethod
     def empty(N: int, K: int, device="cuda", fmt: str = "nf4", scale: str = "e4m3") -> "NF4Weight":
-        nc, n2, n1 = storage_bytes(N, K)
+        nc, n2, n1 = storage_bytes(N, K, scale)
         return NF4Weight(torch.empty(nc, dtype=torch.uint8, device=device),
                          torch.empty(n2, dtype=torch.uint8, device=device),
                          torch.empty(n1 // 4, dtype=torch.float32, device=device), N, K, fmt, scale)

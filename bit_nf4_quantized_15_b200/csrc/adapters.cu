@@ -31,14 +31,16 @@ struct MergeSmem {
   int a, b, codes, chat, out, total;
 };
 
+constexpr int kARow = kMT * 2 + 16;  // L2 tile row (128 n of one j, bytes), padded for ldmatrix
+
 __host__ __device__ inline MergeSmem merge_smem(int rp) {
   MergeSmem s;
-  const int row = (rp + 8) * 2;          // padded adapter row (bytes)
-  s.a = 0;                               // L2^T tile [128 n][rp] bf16
-  s.b = s.a + kMT * row;                 // L1 tile   [128 k][rp] bf16
-  s.codes = s.b + kMT * row;             // [128 n][64] code bytes
+  const int brow = (rp + 8) * 2;         // padded L1 row (bytes)
+  s.a = 0;                               // L2 tile  [rp j][128 n] bf16, as stored in L2
+  s.b = s.a + rp * kARow;                // L1 tile  [128 k][rp] bf16
+  s.codes = s.b + kMT * brow;            // [128 n][64] code bytes
   s.chat = s.codes + kMT * 64;           // c^ [128 n][2 blocks] fp32
-  s.out = 0;                             // [128 n][128 k] bf16 (padded rows), reuses the operand tiles after the MMAs
+  s.out = 0;                             // [128 n][128 k] bf16 (padded rows), reuses the window after the MMAs
   s.total = s.chat + kMT * 2 * 4;
   const int out_bytes = kMT * kOutRow;
   if (s.total < out_bytes) s.total = out_bytes;
@@ -53,56 +55,77 @@ QDEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 fills zeros.
+QDEV void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+QDEV void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Four 8x8 bf16 matrices, transposed on the way: with the row addresses of
+// matrix t/8 in threads 8(t/8) .. 8(t/8)+7, register i of thread t holds
+// elements (2(t%4), t/4) and (2(t%4)+1, t/4) of matrix i as stored.
+QDEV void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
 __global__ void __launch_bounds__(kMThreads) adapter_merge_kernel(const uint8_t* __restrict__ codes,
                                                                    const uint8_t* __restrict__ c2,
-                                                                   const float* __restrict__ c1, int e5m2,
+                                                                   const float* __restrict__ c1, int codec,
                                                                    int64_t N, int64_t K,
                                                                    const uint16_t* __restrict__ L1,
                                                                    const uint16_t* __restrict__ L2, int r, float s,
                                                                    uint16_t* __restrict__ out, Nf4Tables tab) {
   extern __shared__ __align__(16) uint8_t msm[];
   const int rp = (r + 15) & ~15;  // rank padded to whole 16-wide MMA steps (zeros beyond r)
-  const int rowb = (rp + 8) * 2;
+  const int brow = (rp + 8) * 2;
   const MergeSmem L = merge_smem(rp);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n0 = (int64_t)blockIdx.y * kMT, k0 = (int64_t)blockIdx.x * kMT;
   const int nv = (int)min((int64_t)kMT, N - n0), kv = (int)min((int64_t)kMT, K - k0);
+  const uint32_t sbase = smem_u32(msm);
   __shared__ float q[16];
   if (tid < 16) q[tid] = tab.q[tid];
 
-  // ---- stage: L2^T (transposed while staging), L1 rows, codes, block scales
-  for (int i = tid; i < kMT * (rp / 2); i += kMThreads) {  // pairs (j, j+1) of row n
-    const int n = i % kMT, jp = i / kMT, j = 2 * jp;
-    uint32_t v = 0;
-    if (n < nv && j < r) {
-      const uint32_t lo = L2[(int64_t)j * N + n0 + n];
-      const uint32_t hi = j + 1 < r ? L2[(int64_t)(j + 1) * N + n0 + n] : 0u;
-      v = lo | (hi << 16);
-    }
-    *reinterpret_cast<uint32_t*>(msm + L.a + n * rowb + j * 2) = v;
+  // ---- stage with 16-byte asynchronous copies (zero-filled outside the
+  // weight and beyond r): the L2 tile as stored ([j][n], 8 n per piece; N %
+  // 8 == 0 keeps every piece inside or outside the weight), the L1 rows, the
+  // code bytes; then one block scale per thread.
+  for (int i = tid; i < rp * (kMT / 8); i += kMThreads) {
+    const int j = i / (kMT / 8), c = i % (kMT / 8);
+    const bool ok = j < r && c * 8 < nv;
+    cp_async16(sbase + L.a + j * kARow + c * 16, ok ? (const void*)(L2 + (int64_t)j * N + n0 + c * 8) : (const void*)L2,
+               ok ? 16u : 0u);
   }
-  const int vpr = rp / 8;  // 16-byte pieces per padded adapter row
+  const int vpr = rp / 8;  // 16-byte pieces per padded L1 row
   for (int i = tid; i < kMT * vpr; i += kMThreads) {
     const int k = i / vpr, c = i % vpr;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (k < kv && c * 8 < r) v = __ldg(reinterpret_cast<const uint4*>(L1 + (k0 + k) * r) + c);
-    *reinterpret_cast<uint4*>(msm + L.b + k * rowb + c * 16) = v;
+    const bool ok = k < kv && c * 8 < r;
+    cp_async16(sbase + L.b + k * brow + c * 16, ok ? (const void*)(L1 + (k0 + k) * r + c * 8) : (const void*)L1,
+               ok ? 16u : 0u);
   }
   for (int i = tid; i < kMT * 4; i += kMThreads) {  // 64 code bytes per row: four 16-byte pieces
     const int n = i >> 2, c = i & 3;
-    uint4 v = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);
-    if (n < nv && c * 32 < kv) v = __ldg(reinterpret_cast<const uint4*>(codes + ((n0 + n) * K + k0) / 2) + c);
-    *reinterpret_cast<uint4*>(msm + L.codes + n * 64 + c * 16) = v;
+    const bool ok = n < nv && c * 32 < kv;
+    cp_async16(sbase + L.codes + n * 64 + c * 16, ok ? (const void*)(codes + ((n0 + n) * K + k0) / 2 + c * 16)
+                                                     : (const void*)codes,
+               ok ? 16u : 0u);
   }
   {
     const int n = tid >> 1, b = tid & 1;  // 256 threads: one (row, block) scale each
     float ch = 0.0f;
     if (n < nv && b * 64 < kv) {
       const int64_t f = ((n0 + n) * K + k0) / 64 + b;
-      ch = decode_scale(__ldg(c2 + f), __ldg(c1 + (f >> 8)), e5m2 != 0);
+      ch = decode_scale(__ldg(c2 + f), load_group_scale(c1, f >> 8, codec == QLORA_SCALE_E4M3_MEAN),
+                        codec == QLORA_SCALE_E5M2, codec == QLORA_SCALE_E4M3_MEAN);
     }
     reinterpret_cast<float*>(msm + L.chat)[tid] = ch;
   }
+  cp_async_wait_all();
   __syncthreads();
 
   // ---- MMAs: warp (wn, wk) owns rows 64 wn .. +63 and columns 32 wk .. +31
@@ -115,21 +138,19 @@ __global__ void __launch_bounds__(kMThreads) adapter_merge_kernel(const uint8_t*
     for (int b = 0; b < 4; ++b)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.0f;
-  const uint8_t* As = msm + L.a + (64 * wn) * rowb;
-  const uint8_t* Bs = msm + L.b + (32 * wk) * rowb;
+  // A = L2^T (rows n, reduction j) by transposing loads of the [j][n] tile:
+  // matrix mq of a 16 x 16 step = rows n + 8 (mq & 1), reduction j + 8 (mq >> 1).
+  const int mq = lane >> 3, mr = lane & 7;
+  const uint32_t a_lane = sbase + L.a + (uint32_t)(((mq >> 1) * 8 + mr) * kARow + (64 * wn + (mq & 1) * 8) * 2);
+  const uint8_t* Bs = msm + L.b + (32 * wk) * brow;
   for (int j0 = 0; j0 < rp; j0 += 16) {
     uint32_t af[4][4], bfr[4][2];
 #pragma unroll
-    for (int mi = 0; mi < 4; ++mi) {
-      const uint8_t* p = As + (16 * mi + gr) * rowb + (j0 + 2 * cq) * 2;
-      af[mi][0] = *reinterpret_cast<const uint32_t*>(p);
-      af[mi][1] = *reinterpret_cast<const uint32_t*>(p + 8 * rowb);
-      af[mi][2] = *reinterpret_cast<const uint32_t*>(p + 16);
-      af[mi][3] = *reinterpret_cast<const uint32_t*>(p + 8 * rowb + 16);
-    }
+    for (int mi = 0; mi < 4; ++mi)
+      ldmatrix_x4_trans(a_lane + (uint32_t)(j0 * kARow + mi * 32), af[mi][0], af[mi][1], af[mi][2], af[mi][3]);
 #pragma unroll
     for (int ni = 0; ni < 4; ++ni) {
-      const uint8_t* p = Bs + (8 * ni + gr) * rowb + (j0 + 2 * cq) * 2;
+      const uint8_t* p = Bs + (8 * ni + gr) * brow + (j0 + 2 * cq) * 2;
       bfr[ni][0] = *reinterpret_cast<const uint32_t*>(p);
       bfr[ni][1] = *reinterpret_cast<const uint32_t*>(p + 16);
     }
@@ -247,8 +268,8 @@ cudaError_t launch_adapter_merge(const uint8_t* codes, const uint8_t* c2, const 
   cudaError_t err = cudaFuncSetAttribute(adapter_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((K + kMT - 1) / kMT), (unsigned)((N + kMT - 1) / kMT));
-  adapter_merge_kernel<<<grid, kMThreads, smem, st>>>(codes, c2, c1, scale_codec == QLORA_SCALE_E5M2, N, K, L1, L2, r,
-                                                       s, out, code_tables(format));
+  adapter_merge_kernel<<<grid, kMThreads, smem, st>>>(codes, c2, c1, scale_codec, N, K, L1, L2, r, s, out,
+                                                       code_tables(format));
   count_launches(1);
   return cudaGetLastError();
 }

@@ -70,6 +70,24 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize
   return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// 3-D map over a row-major matrix [rows][cols] of bf16 viewed as
+// (64, rows, cols / 64): element (x, y, z) is [y][64 z + x]; box 64 x
+// box_rows x box_blocks, 128-byte swizzle.  One load brings box_blocks
+// consecutive 64-wide column blocks of box_rows rows.
+int map_blocks3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                 uint32_t box_blocks) {
+  auto fn = encode_fn();
+  if (!fn) return QLORA_ERR_CUDA;
+  const cuuint64_t dims[3] = {64, rows, cols / 64};
+  const cuuint64_t strides[2] = {cols * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, box_blocks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // bf16 operand of the engine.  K-major: matrix [mn][k] (k contiguous), box
 // 64 k x `rows` mn.  MN-major: matrix [k][mn] (mn contiguous), box 64 x 64.
 int map_operand(CUtensorMap* m, const void* base, int mn_major, uint64_t mn_extent, uint64_t k_extent, int rows) {
@@ -101,13 +119,21 @@ EpiArgs epi_none() {
 }
 
 bool format_ok(const qlora_nf4_weight* w) {
-  return w->format >= 0 && w->format < kNumFormats && (w->scale_codec == QLORA_SCALE_E4M3 || w->scale_codec == QLORA_SCALE_E5M2);
+  return w->format >= 0 && w->format < kNumFormats &&
+         (w->scale_codec == QLORA_SCALE_E4M3 || w->scale_codec == QLORA_SCALE_E5M2 ||
+          w->scale_codec == QLORA_SCALE_E4M3_MEAN);
+}
+
+// The mean-centred codec reads [c1, mean] pairs as 8-byte loads.
+bool c1_aligned(const qlora_nf4_weight* w) {
+  return w->scale_codec != QLORA_SCALE_E4M3_MEAN || (reinterpret_cast<uintptr_t>(w->c1) & 7u) == 0;
 }
 
 void fill_common(EngineArgs* a, int* status, int format, int scale_codec) {
   std::memset(a, 0, sizeof(*a));
   a->status = status;
   a->c2_e5m2 = scale_codec == QLORA_SCALE_E5M2;
+  a->c1_mean = scale_codec == QLORA_SCALE_E4M3_MEAN;
   const Nf4Tables& t = code_tables(format);
   for (int i = 0; i < 16; ++i) a->q[i] = t.q[i];
 }
@@ -222,13 +248,20 @@ const char* qlora_status_string(int code) {
   return "unknown status";
 }
 
-int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes, size_t* c2_bytes, size_t* c1_bytes) {
+int qlora_weight_storage_bytes(int64_t N, int64_t K, int scale_codec, size_t* codes_bytes, size_t* c2_bytes,
+                               size_t* c1_bytes) {
   if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
+  if (scale_codec != QLORA_SCALE_E4M3 && scale_codec != QLORA_SCALE_E5M2 && scale_codec != QLORA_SCALE_E4M3_MEAN)
+    return QLORA_ERR_FORMAT;
   const int64_t n = N * K, nb = n / 64;
   if (codes_bytes) *codes_bytes = (size_t)(n / 2);
   if (c2_bytes) *c2_bytes = (size_t)nb;
-  if (c1_bytes) *c1_bytes = (size_t)((nb + 255) / 256) * 4;
+  if (c1_bytes) *c1_bytes = (size_t)((nb + 255) / 256) * (scale_codec == QLORA_SCALE_E4M3_MEAN ? 8 : 4);
   return QLORA_OK;
+}
+
+int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes, size_t* c2_bytes, size_t* c1_bytes) {
+  return qlora_weight_storage_bytes(N, K, QLORA_SCALE_E4M3, codes_bytes, c2_bytes, c1_bytes);
 }
 
 uint64_t qlora_kernel_launches(void) { return launches_so_far(); }
@@ -264,6 +297,7 @@ int qlora_nf4_quantize(const uint16_t* W, int64_t N, int64_t K, const qlora_nf4_
   if (!W || !out || !out->codes || !out->c2 || !out->c1) return QLORA_ERR_NULL;
   if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
   if (!format_ok(out)) return QLORA_ERR_FORMAT;
+  if (!c1_aligned(out)) return QLORA_ERR_ALIGN;
   if (!aligned16(W) || !aligned16(out->codes)) return QLORA_ERR_ALIGN;
   DevInfo di;
   if (int rc = current_device_info(&di)) return rc;
@@ -279,6 +313,7 @@ int qlora_nf4_dequant(const qlora_nf4_weight* w, uint16_t* W_out, int* status_de
   if (!w || !W_out || !w->codes || !w->c2 || !w->c1) return QLORA_ERR_NULL;
   if (w->n_rows < 1 || w->n_cols < 64 || w->n_cols % 64) return QLORA_ERR_SHAPE;
   if (!format_ok(w)) return QLORA_ERR_FORMAT;
+  if (!c1_aligned(w)) return QLORA_ERR_ALIGN;
   if (!aligned16(W_out) || !aligned16(w->codes)) return QLORA_ERR_ALIGN;
   DevInfo di;
   if (int rc = current_device_info(&di)) return rc;
@@ -303,6 +338,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
   const int64_t N = w->n_rows, K = w->n_cols;
   if (!shape_ok(M, N, K)) return QLORA_ERR_SHAPE;
   if (!format_ok(w)) return QLORA_ERR_FORMAT;
+  if (!c1_aligned(w)) return QLORA_ERR_ALIGN;
   if (!valid_rank(r)) return QLORA_ERR_RANK;
   for (const void* p : {(const void*)X, (const void*)w->codes, (const void*)L1, (const void*)L2, (const void*)Y,
                         (const void*)T_save, (const void*)ws})
@@ -323,7 +359,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
     std::memset(&ga, 0, sizeof(ga));
     if (make_map(&ga.tmCodes, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 128, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        map_operand(&ga.tmX, X, 0, M, K, 16))
+        map_blocks3d(&ga.tmX, X, (uint64_t)M, (uint64_t)K, 16, 4))
       return QLORA_ERR_CUDA;
     ga.c2 = w->c2;
     ga.c1 = w->c1;
@@ -345,6 +381,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, co
     ga.status = status_dev;
     const Nf4Tables& tb = code_tables(w->format);
     ga.c2_e5m2 = w->scale_codec == QLORA_SCALE_E5M2;
+    ga.c1_mean = w->scale_codec == QLORA_SCALE_E4M3_MEAN;
     for (int i = 0; i < 16; ++i) ga.q[i] = tb.q[i];
     cudaEvent_t e0 = g_ev_start, e1 = g_ev_end;
     g_ev_start = g_ev_end = nullptr;
@@ -412,6 +449,7 @@ int qlora_adapter_merge(const qlora_nf4_weight* w, const uint16_t* L1, const uin
   const int64_t N = w->n_rows, K = w->n_cols;
   if (!shape_ok(1, N, K)) return QLORA_ERR_SHAPE;
   if (!format_ok(w)) return QLORA_ERR_FORMAT;
+  if (!c1_aligned(w)) return QLORA_ERR_ALIGN;
   if (!valid_rank(r)) return QLORA_ERR_RANK;
   for (const void* p : {(const void*)w->codes, (const void*)L1, (const void*)L2, (const void*)W_out})
     if (!aligned16(p)) return QLORA_ERR_ALIGN;
@@ -470,6 +508,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const flo
   const int64_t N = w->n_rows, K = w->n_cols;
   if (!shape_ok(M, N, K)) return QLORA_ERR_SHAPE;
   if (!format_ok(w)) return QLORA_ERR_FORMAT;
+  if (!c1_aligned(w)) return QLORA_ERR_ALIGN;
   if (!valid_rank(r)) return QLORA_ERR_RANK;
   for (const void* p : {(const void*)dY, (const void*)X, (const void*)T_saved, (const void*)w->codes,
                         (const void*)L1, (const void*)L2, (const void*)ws})

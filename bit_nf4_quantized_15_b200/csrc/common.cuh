@@ -128,6 +128,15 @@ QDEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int
       : "memory");
 }
 
+// 3-D tiled load (x innermost, then y, then z), completion on `bar`.
+QDEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // ------------------------------------------------------------------- tcgen05
 QDEV void tmem_alloc(uint32_t* slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
@@ -227,10 +236,26 @@ QDEV float e4m3_to_float(uint32_t code) {
 // same value).
 QDEV float e5m2_to_float(uint32_t code) { return __half2float(__ushort_as_half((unsigned short)(code << 8))); }
 
+// Second-level scale of a group of 256 blocks: c1 and, for the mean-centred
+// codec (QLORA_SCALE_E4M3_MEAN, whose c1 array holds [c1, mean] pairs), the
+// group mean of the block scales.
+struct GroupScale {
+  float c1, mu;
+};
+QDEV GroupScale load_group_scale(const float* c1, int64_t g, bool mean) {
+  if (mean) {
+    const float2 v = __ldg(reinterpret_cast<const float2*>(c1) + g);
+    return GroupScale{v.x, v.y};
+  }
+  return GroupScale{__ldg(c1 + g), 0.0f};
+}
+
 // Decoded block scale c^ = RN32(dec(c2) * c1); c2 is E4M3, or E5M2 for the
-// scale-codec variant.
-QDEV float decode_scale(uint32_t c2code, float c1v, bool e5m2 = false) {
-  return __fmul_rn(e5m2 ? e5m2_to_float(c2code) : e4m3_to_float(c2code), c1v);
+// scale-codec variant; the mean-centred codec adds the group mean with a
+// second rounding, RN32(RN32(dec(c2) * c1) + mean) (signed E4M3 residual).
+QDEV float decode_scale(uint32_t c2code, GroupScale gs, bool e5m2, bool mean) {
+  const float p = __fmul_rn(e5m2 ? e5m2_to_float(c2code) : e4m3_to_float(c2code), gs.c1);
+  return mean ? __fadd_rn(p, gs.mu) : p;
 }
 
 QDEV uint32_t pack_bf16x2(float lo, float hi) {

@@ -229,22 +229,22 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
       const uint32_t tlane = tmem_d + ((uint32_t)(q4 * 32) << 16) + TM::a_col;
       const int sw = (rl >> 2) & 1;  // 32-byte swizzle of the code tile
       uint32_t c2raw = 0;
-      float c1v = 0.0f;
+      GroupScale gsc{0.0f, 0.0f};
       if (valid && grp < my_kb) {
         const int64_t f = n * bpr + kb_lo + grp;
         c2raw = __ldg(args.c2 + f);
-        c1v = __ldg(args.c1 + (f >> 8));
+        gsc = load_group_scale(args.c1, f >> 8, args.c1_mean != 0);
       }
       for (int it = grp; it < my_kb; it += R::G) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const uint32_t taddr = tlane + (uint32_t)(s * 32);
         const uint8_t* ctile = smem + s * L::STAGE + kA + L::B + rl * 32;
-        const float chat = valid ? decode_scale(c2raw, c1v, args.c2_e5m2 != 0) : 0.0f;
+        const float chat = valid ? decode_scale(c2raw, gsc, args.c2_e5m2 != 0, args.c1_mean != 0) : 0.0f;
         if (valid && it + R::G < my_kb) {  // this group's next scale, one round ahead
           const int64_t f = n * bpr + kb_lo + it + R::G;
           c2raw = __ldg(args.c2 + f);
-          c1v = __ldg(args.c1 + (f >> 8));
+          gsc = load_group_scale(args.c1, f >> 8, args.c1_mean != 0);
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
         if (!warp_wait(empty + s, ph ^ 1u, abort_flag, args.status, lane, lim)) break;
@@ -282,28 +282,28 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
       const uint8_t* ctile = sa + kA + L::B + nl * 64;
       uint8_t* atile = sa + mb * 8192 + (nl >> 3) * 1024 + r8 * 128;
       uint32_t c2raw = 0;
-      float c1v = 0.0f;
+      GroupScale gsc{0.0f, 0.0f};
       {
         const int64_t nn = (int64_t)(kb_lo + grp) * 64 + nl;
         if (kvalid && nn < args.wN && grp < my_kb) {
           const int64_t f = nn * bpr + kblk;
           c2raw = __ldg(args.c2 + f);
-          c1v = __ldg(args.c1 + (f >> 8));
+          gsc = load_group_scale(args.c1, f >> 8, args.c1_mean != 0);
         }
       }
       for (int it = grp; it < my_kb; it += kStages) {
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const int64_t nn = (int64_t)(kb_lo + it) * 64 + nl;
         const bool valid = kvalid && nn < args.wN;
-        const float chat = valid ? decode_scale(c2raw, c1v, args.c2_e5m2 != 0) : 0.0f;
+        const float chat = valid ? decode_scale(c2raw, gsc, args.c2_e5m2 != 0, args.c1_mean != 0) : 0.0f;
         if (it + kStages < my_kb) {
           const int64_t nx = nn + 64 * kStages;
           c2raw = 0;
-          c1v = 0.0f;
+          gsc = GroupScale{0.0f, 0.0f};
           if (kvalid && nx < args.wN) {
             const int64_t f = nx * bpr + kblk;
             c2raw = __ldg(args.c2 + f);
-            c1v = __ldg(args.c1 + (f >> 8));
+            gsc = load_group_scale(args.c1, f >> 8, args.c1_mean != 0);
           }
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);

@@ -298,27 +298,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       const uint32_t tlane = tmem_d + ((uint32_t)(q4 * 32) << 16) + kPAcc;
       const uint4* crow = reinterpret_cast<const uint4*>(args.codes + (valid ? n : 0) * (args.wK / 2));
       uint32_t c2raw = 0;
-      float c1v = 0.0f;
+      GroupScale gsc{0.0f, 0.0f};
       uint4 cn0 = make_uint4(0, 0, 0, 0), cn1 = cn0;  // this group's next code block (k 0..31, 32..63)
       if (valid && grp < n_kb) {
         const int64_t f = n * bpr + grp;
         cn0 = __ldg(crow + 2 * grp);
         cn1 = __ldg(crow + 2 * grp + 1);
         c2raw = __ldg(args.c2 + f);
-        c1v = __ldg(args.c1 + (f >> 8));
+        gsc = load_group_scale(args.c1, f >> 8, args.c1_mean != 0);
       }
       for (int it = grp; it < n_kb; it += kPG) {
         const int a = it % kPA;
         const uint32_t ph = (uint32_t)(it / kPA) & 1u;
         const uint32_t taddr = tlane + (uint32_t)(a * 32);
         const uint4 c0 = cn0, c1 = cn1;
-        const float chat = valid ? decode_scale(c2raw, c1v, args.c2_e5m2 != 0) : 0.0f;
+        const float chat = valid ? decode_scale(c2raw, gsc, args.c2_e5m2 != 0, args.c1_mean != 0) : 0.0f;
         if (valid && it + kPG < n_kb) {  // this group's next codes and scale, one round ahead
           const int64_t f = n * bpr + it + kPG;
           cn0 = __ldg(crow + 2 * (it + kPG));
           cn1 = __ldg(crow + 2 * (it + kPG) + 1);
           c2raw = __ldg(args.c2 + f);
-          c1v = __ldg(args.c1 + (f >> 8));
+          gsc = load_group_scale(args.c1, f >> 8, args.c1_mean != 0);
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
         if (!warp_wait(aempty + a, ph ^ 1u, abort_flag, args.status, lane)) break;

@@ -56,7 +56,7 @@ constexpr int kWS = 2;                     // ring stages per worker
 constexpr int kNS = kWG * kWS;             // stages per CTA
 constexpr int kUnitKB = 4;                 // 64-wide k blocks per unit
 constexpr int kCodeBytes = 16384;          // 128 rows x 128 bytes (256 codes)
-constexpr int kXBytes = 8192;              // 16 tokens x 256 bf16 (4 boxes of 64)
+constexpr int kXBytes = 8192;              // 16 tokens x 256 bf16: one 3-D box of 4 x (16 x 64)
 constexpr int kStageBytes = kCodeBytes + kXBytes;
 // A worker's warps each own kRG 16-row groups of the 128-row tile.
 constexpr int kRG = 2;
@@ -158,20 +158,29 @@ QDEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :
 // block (four consecutive blocks cross at most one 256-block group).
 struct RowScales {
   uint32_t c2;
-  float c1a, c1b;
+  GroupScale ga, gb;  // groups of the unit's first and last block
 };
+// Issued one unit ahead of use.  The four codes come as one 32-bit load
+// when they are 4-byte aligned (K a multiple of 256 makes every row's unit
+// aligned), so no instruction consumes the loaded values before the next
+// unit: packing bytes right after their loads would stall the warp for the
+// whole memory latency at the prefetch.
 QDEV RowScales load_row_scales(const GemvArgs& a, int rt, int un, int rl) {
-  RowScales s{0u, 0.0f, 0.0f};
+  RowScales s{0u, GroupScale{0.0f, 0.0f}, GroupScale{0.0f, 0.0f}};
   const int64_t n = (int64_t)rt * 128 + rl;
   if (n >= a.N) return s;
   const int kb0 = un * kUnitKB;
   const int64_t f0 = n * a.kbt + kb0;
   const int nkb = min(kUnitKB, a.kbt - kb0);
+  if (nkb == kUnitKB && (f0 & 3) == 0) {
+    s.c2 = __ldg(reinterpret_cast<const uint32_t*>(a.c2 + f0));
+  } else {
 #pragma unroll
-  for (int q = 0; q < kUnitKB; ++q)
-    if (q < nkb) s.c2 |= (uint32_t)__ldg(a.c2 + f0 + q) << (8 * q);
-  s.c1a = __ldg(a.c1 + (f0 >> 8));
-  s.c1b = __ldg(a.c1 + ((f0 + nkb - 1) >> 8));
+    for (int q = 0; q < kUnitKB; ++q)
+      if (q < nkb) s.c2 |= (uint32_t)__ldg(a.c2 + f0 + q) << (8 * q);
+  }
+  s.ga = load_group_scale(a.c1, f0 >> 8, a.c1_mean != 0);
+  s.gb = load_group_scale(a.c1, (f0 + nkb - 1) >> 8, a.c1_mean != 0);
   return s;
 }
 // c^ = RN32(dec(c2) . c1) of the unit's four k blocks for one row, whose
@@ -179,7 +188,7 @@ QDEV RowScales load_row_scales(const GemvArgs& a, int rt, int un, int rl) {
 // (f0 mod 256) + q >= 256).  Two codes per conversion: an E4M3 pair through
 // the hardware fp8x2 -> f16x2 conversion, an E5M2 byte as the high byte of
 // an fp16; both exact.
-QDEV void row_chats(const RowScales& s, int64_t f0, bool e5m2, float (&out)[kUnitKB]) {
+QDEV void row_chats(const RowScales& s, int64_t f0, bool e5m2, bool mean, float (&out)[kUnitKB]) {
   float2 v01, v23;
   if (e5m2) {
     const uint32_t b01 = __byte_perm(s.c2, 0u, 0x1404u), b23 = __byte_perm(s.c2, 0u, 0x3424u);
@@ -192,10 +201,13 @@ QDEV void row_chats(const RowScales& s, int64_t f0, bool e5m2, float (&out)[kUni
     v23 = __half22float2(__half2(h23));
   }
   const int g0 = (int)(f0 & 255);
-  out[0] = __fmul_rn(v01.x, g0 + 0 < 256 ? s.c1a : s.c1b);
-  out[1] = __fmul_rn(v01.y, g0 + 1 < 256 ? s.c1a : s.c1b);
-  out[2] = __fmul_rn(v23.x, g0 + 2 < 256 ? s.c1a : s.c1b);
-  out[3] = __fmul_rn(v23.y, g0 + 3 < 256 ? s.c1a : s.c1b);
+  const float v[kUnitKB] = {v01.x, v01.y, v23.x, v23.y};
+#pragma unroll
+  for (int q = 0; q < kUnitKB; ++q) {
+    const GroupScale& gs = g0 + q < 256 ? s.ga : s.gb;
+    const float p = __fmul_rn(v[q], gs.c1);
+    out[q] = mean ? __fadd_rn(p, gs.mu) : p;  // mean-centred codec: + group mean, rounded again
+  }
 }
 
 // NT = 8-token column tiles (1 for M <= 8, 2 for M <= 16).
@@ -247,13 +259,12 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
           break;
         const int64_t u = u0 + i;
         const int rt = (int)(u / upr), un = (int)(u % upr);
-        const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);  // k blocks of W in this unit
         const uint32_t st = stage_addr(S, kWS * g + j);
         uint8_t* sp = S.raw + (st - S.raw_addr);
-        mbar_arrive_expect_tx(bar_full(S, g, j), kCodeBytes + (uint32_t)nkb * 2048u);
+        mbar_arrive_expect_tx(bar_full(S, g, j), kCodeBytes + kXBytes);
         tma_load_2d(sp, &args.tmCodes, bar_full(S, g, j), un * 128, rt * 128);
-        for (int q = 0; q < nkb; ++q)
-          tma_load_2d(sp + kCodeBytes + q * 2048, &args.tmX, bar_full(S, g, j), (un * kUnitKB + q) * 64, 0);
+        // the unit's four 64-wide X blocks in one box (blocks beyond K read as zeros)
+        tma_load_3d(sp + kCodeBytes, &args.tmX, bar_full(S, g, j), 0, 0, un * kUnitKB);
         issued = i + 1;
       }
       if (*S.abort_flag) {  // let the loads already issued land before exit
@@ -316,7 +327,8 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
       float chs[2 * kRG][kUnitKB];  // c^ of this unit's blocks, per thread row
 #pragma unroll
       for (int r = 0; r < 2 * kRG; ++r)
-        row_chats(sc[r], ((int64_t)rt * 128 + rows[r]) * args.kbt + (int64_t)un * kUnitKB, args.c2_e5m2 != 0, chs[r]);
+        row_chats(sc[r], ((int64_t)rt * 128 + rows[r]) * args.kbt + (int64_t)un * kUnitKB, args.c2_e5m2 != 0,
+                  args.c1_mean != 0, chs[r]);
       if (i + 1 < nu) {
 #pragma unroll
         for (int r = 0; r < 2 * kRG; ++r) sc[r] = load_row_scales(args, (int)((u + 1) / upr), (int)((u + 1) % upr), rows[r]);

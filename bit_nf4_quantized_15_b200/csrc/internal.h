@@ -67,6 +67,7 @@ struct EngineArgs {
   const uint8_t* codes;  // NF4 codes [wN][wK/2] (read directly by the pair forward)
   const uint8_t* c2;
   int c2_e5m2;           // c2 holds E5M2 codes instead of E4M3
+  int c1_mean;           // mean-centred codec: c1 holds [c1, mean] per group
   const float* c1;
   int64_t wN, wK;    // quantised weight shape (for scale indexing)
   int rows, cols;    // output extent: UMMA-M side, UMMA-N side
@@ -130,9 +131,10 @@ struct GemvPlan {
 
 struct GemvArgs {
   CUtensorMap tmCodes;  // uint8 [N][K/2], box 128 x 128, 128-byte swizzle
-  CUtensorMap tmX;      // bf16 [M][K], box 64 x 16, 128-byte swizzle
+  CUtensorMap tmX;      // bf16 [M][K] as 3-D (64, M, K/64), box 64 x 16 x 4, 128-byte swizzle
   const uint8_t* c2;
   int c2_e5m2;          // c2 holds E5M2 codes instead of E4M3
+  int c1_mean;          // mean-centred codec: c1 holds [c1, mean] per group
   const float* c1;
   int64_t N, K;
   int M;

@@ -98,10 +98,12 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
                                                                       uint2* __restrict__ codes,
                                                                       uint8_t* __restrict__ c2,
                                                                       float* __restrict__ c1, int* status,
-                                                                      QuantParams qp, int e5m2) {
+                                                                      QuantParams qp, int codec) {
   __shared__ float s_t[16];
   __shared__ float s_absmax[kGroupBlocks];
   __shared__ float s_wmax[kQuantThreads / 32];
+  __shared__ float s_wsum[kQuantThreads / 32];
+  const bool e5m2 = codec == QLORA_SCALE_E5M2, mean = codec == QLORA_SCALE_E4M3_MEAN;
   const int t = threadIdx.x;
   if (t < 16) s_t[t] = t < 15 ? qp.t[t] : 2.0f;
   float2 P[6];
@@ -172,9 +174,25 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
     if (__any_sync(0xFFFFFFFFu, bad) && (t & 31) == 0) report(status, QLORA_ERR_NONFINITE);
     __syncthreads();
     // second level: c1 = RN32(max c_b / 448), c2_b = E4M3(RN32(c_b / c1));
-    // for E5M2 scale codes 57344 and E5M2
-    float cb = t < nblk ? s_absmax[t] : 0.0f;
-    float wm = cb;
+    // for E5M2 scale codes 57344 and E5M2.  Mean-centred: the group mean mu
+    // (fp32 pairwise tree over the 256 slots, empty slots zero: the butterfly
+    // of lane sums, then the eight warp sums pairwise), d_b = RN32(c_b - mu),
+    // c1 = RN32(max |d_b| / 448), signed E4M3 codes of RN32(d_b / c1).
+    const float cb = t < nblk ? s_absmax[t] : 0.0f;
+    float d = cb, mu = 0.0f;
+    if (mean) {
+      float sum = cb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
+      if ((t & 31) == 0) s_wsum[t >> 5] = sum;
+      __syncthreads();
+      const float s01 = __fadd_rn(s_wsum[0], s_wsum[1]), s23 = __fadd_rn(s_wsum[2], s_wsum[3]);
+      const float s45 = __fadd_rn(s_wsum[4], s_wsum[5]), s67 = __fadd_rn(s_wsum[6], s_wsum[7]);
+      const float total = __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67));
+      mu = __fdiv_rn(total, (float)nblk);
+      d = t < nblk ? __fsub_rn(cb, mu) : 0.0f;
+    }
+    float wm = fabsf(d);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xFFFFFFFFu, wm, o));
     if ((t & 31) == 0) s_wmax[t >> 5] = wm;
@@ -183,11 +201,14 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
 #pragma unroll
     for (int k = 1; k < kQuantThreads / 32; ++k) gmax = fmaxf(gmax, s_wmax[k]);
     const float c1v = __fdiv_rn(gmax, e5m2 ? 57344.0f : 448.0f);
-    if (t == 0) c1[g] = c1v;
+    if (t == 0) {
+      if (mean) reinterpret_cast<float2*>(c1)[g] = make_float2(c1v, mu);
+      else c1[g] = c1v;
+    }
     if (t < nblk) {
       uint8_t code = 0;
       if (c1v > 0.0f)
-        code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(cb, c1v), __NV_SATFINITE, e5m2 ? __NV_E5M2 : __NV_E4M3);
+        code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(d, c1v), __NV_SATFINITE, e5m2 ? __NV_E5M2 : __NV_E4M3);
       c2[blk0 + t] = code;
     }
     __syncthreads();
@@ -203,7 +224,8 @@ constexpr int kDeqSteps = 8;
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ codes,
                                                           const uint8_t* __restrict__ c2,
                                                           const float* __restrict__ c1, int64_t n_chunks,
-                                                          uint4* __restrict__ out, Nf4Tables tab, int e5m2) {
+                                                          uint4* __restrict__ out, Nf4Tables tab, int codec) {
+  const bool e5m2 = codec == QLORA_SCALE_E5M2, mean = codec == QLORA_SCALE_E4M3_MEAN;
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = tab.q[threadIdx.x];
   __syncthreads();
@@ -211,7 +233,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __rest
   for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < n_chunks; c0 += kDeqSteps * stride) {
     uint32_t cw[kDeqSteps];
     uint32_t s2[kDeqSteps];
-    float s1[kDeqSteps];
+    GroupScale s1[kDeqSteps];
 #pragma unroll
     for (int u = 0; u < kDeqSteps; ++u) {
       const int64_t ci = c0 + u * stride;
@@ -219,14 +241,14 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __rest
         cw[u] = __ldcs(codes + ci);
         const int64_t blk = ci >> 3;
         s2[u] = __ldg(c2 + blk);
-        s1[u] = __ldg(c1 + (blk >> 8));
+        s1[u] = load_group_scale(c1, blk >> 8, mean);
       }
     }
 #pragma unroll
     for (int u = 0; u < kDeqSteps; ++u) {
       const int64_t ci = c0 + u * stride;
       if (ci < n_chunks) {
-        const float chat = decode_scale(s2[u], s1[u], e5m2 != 0);
+        const float chat = decode_scale(s2[u], s1[u], e5m2, mean);
         const float2 cc = make_float2(chat, chat);
         uint32_t o[4];
 #pragma unroll

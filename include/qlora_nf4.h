@@ -89,8 +89,23 @@ enum {
  */
 enum {
   QLORA_SCALE_E4M3 = 0,
-  QLORA_SCALE_E5M2 = 1
+  QLORA_SCALE_E5M2 = 1,
+  QLORA_SCALE_E4M3_MEAN = 2
 };
+
+/*
+ * QLORA_SCALE_E4M3_MEAN: mean-centred double quantisation.  The block scales
+ * are all non-negative, so each group of 256 is centred on its mean first and
+ * the signed residuals take the sign bit of E4M3:
+ *   mu_g = RN32(S_g / n_g), S_g the fp32 sum of the group's c_b as a pairwise
+ *          tree over 256 slots (adjacent pairs first; empty slots of a partial
+ *          group are zeros), n_g its number of blocks
+ *   d_b  = RN32(c_b - mu_g);  c1_g = RN32(max |d_b| / 448)
+ *   c2_b = E4M3_RNE_satfinite(RN32(d_b / c1_g)) (signed), 0 when c1_g = 0
+ *   c^_b = RN32(RN32(dec(c2_b) * c1_g) + mu_g)
+ * The c1 array then holds two floats per group, c1_g then mu_g (8-byte
+ * aligned): 4 + 8/64 + 64/16384 bits per weight.  Codes are unchanged.
+ */
 
 /*
  * The quantized weight (nlp-lineage "QLoRA", section "The idea": blocks of
@@ -114,9 +129,15 @@ typedef struct qlora_nf4_weight {
 } qlora_nf4_weight;
 
 /* Bytes of codes, c2 and c1 for an N x K weight (sizes for the caller's
- * allocations).  Returns QLORA_ERR_SHAPE for an invalid shape. */
+ * allocations) with E4M3 or E5M2 block scales.  Returns QLORA_ERR_SHAPE for
+ * an invalid shape. */
 QLORA_API int qlora_nf4_storage_bytes(int64_t N, int64_t K, size_t* codes_bytes, size_t* c2_bytes,
                             size_t* c1_bytes);
+
+/* The same for any scale codec (QLORA_SCALE_*): the mean-centred codec
+ * stores two floats per group in c1.  QLORA_ERR_FORMAT for an unknown codec. */
+QLORA_API int qlora_weight_storage_bytes(int64_t N, int64_t K, int scale_codec, size_t* codes_bytes,
+                                         size_t* c2_bytes, size_t* c1_bytes);
 
 /* The 16 NF4 levels the kernels use (ascending, -1 ... 0 ... 1), copied to a
  * host array.  The library derives them at load from the normal quantiles:

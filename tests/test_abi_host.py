@@ -117,7 +117,7 @@ def test_format_checks_before_any_launch(q):
     fake = P(0x10000)
     arr = (ctypes.c_float * 16)()
     assert L.qlora_code_levels(3, arr) == -11 and L.qlora_code_levels(-1, arr) == -11
-    for fmt, res in ((3, 0), (0, 2), (0, -1)):
+    for fmt, res in ((3, 0), (0, 3), (0, -1)):
         w = q.qlora_nf4_weight(0x1000, 0x2000, 0x3000, 64, 128, fmt, res)
         assert L.qlora_nf4_quantize(fake, 64, 128, ctypes.byref(w), None, None) == -11
         assert L.qlora_nf4_dequant(ctypes.byref(w), fake, None, None) == -11
@@ -151,3 +151,17 @@ def test_adapter_entry_points_check_arguments_before_any_launch(q):
     assert L.qlora_adamw_step(fake, None, fake, fake, fake, 0, pc, None) == 0      # nothing to do
     assert L.qlora_paged_alloc(16, None) == -1 and L.qlora_paged_prefetch(None, 16, 0, None) == -1
     assert L.qlora_paged_free(None) == 0
+
+
+def test_storage_bytes_per_scale_codec(q):
+    """The mean-centred codec stores [c1, mean] per group of 256 blocks."""
+    assert q.storage_bytes(4096, 4096, "e4m3") == (4096 * 4096 // 2, 4096 * 4096 // 64, 4096 * 4096 // 16384 * 4)
+    assert q.storage_bytes(4096, 4096, "e5m2") == q.storage_bytes(4096, 4096)
+    assert q.storage_bytes(4096, 4096, "e4m3_mean")[2] == 2 * q.storage_bytes(4096, 4096)[2]
+    assert q.storage_bytes(3, 128, "e4m3_mean")[2] == 8                      # one partial group
+    L = q.lib()
+    a = ctypes.c_size_t()
+    assert L.qlora_weight_storage_bytes(64, 128, 3, ctypes.byref(a), None, None) == -11
+    P = ctypes.c_void_p
+    w = q.qlora_nf4_weight(0x1000, 0x2000, 0x3004, 64, 128, 0, 2)          # [c1, mean] pairs need 8 bytes
+    assert L.qlora_nf4_dequant(ctypes.byref(w), P(0x10000), None, None) == -2

@@ -105,14 +105,15 @@ def test_pair_forward_parity(lib, monkeypatch, M, N, K, r, pair):
         assert_close(got[k], ref[k], f"{k} M={M} N={N} K={K} r={r} pair={pair}")
 
 
-# The compared 4-bit formats and the E5M2 scale codec through every kernel
-# that dequantises on chip:
+# The compared 4-bit formats and the E5M2 and mean-centred scale codecs
+# through every kernel that dequantises on chip:
 # the forward and dX engines (with a split reduction and without), the
 # few-token GEMV path and the opt-in CTA-pair forward.
 FORMAT_SHAPES = [(300, 256, 192, 16, "0"), (2048, 4096, 512, 32, "1"), (7, 1000, 704, 32, "0")]
 
 
-@pytest.mark.parametrize("fmt,scale", [("fp4", "e4m3"), ("int4", "e4m3"), ("nf4", "e5m2"), ("int4", "e5m2")])
+@pytest.mark.parametrize("fmt,scale", [("fp4", "e4m3"), ("int4", "e4m3"), ("nf4", "e5m2"), ("int4", "e5m2"),
+                                       ("nf4", "e4m3_mean"), ("fp4", "e4m3_mean")])
 @pytest.mark.parametrize("M,N,K,r,pair", FORMAT_SHAPES)
 def test_formats_linear_parity(lib, monkeypatch, fmt, scale, M, N, K, r, pair):
     monkeypatch.setenv("QLORA_NF4_PAIR", pair)

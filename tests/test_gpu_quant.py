@@ -199,6 +199,51 @@ def test_e5m2_scales_every_significand_pair(lib):
     assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, *Wb.shape, scale="e5m2"))
 
 
+# --------------- scale codec variant: E4M3 residuals from each group's mean
+@pytest.mark.parametrize("fmt", ["nf4", "int4"])
+@pytest.mark.parametrize("N,K,seed", [(1, 64, 30), (3, 128, 31), (37, 64 * 300, 32), (256, 4096, 33),
+                                      (8, 16384 * 3, 34)])
+def test_mean_scales_quantize_dequant_bitexact(lib, fmt, N, K, seed):
+    """Group mean (fp32 pairwise tree), signed E4M3 residual codes, [c1, mean]
+    pairs and the dequantised weights, bit for bit; partial last groups and
+    one-block groups included."""
+    Wb = mixed_weights(N, K, seed)
+    ref = O.quantize(Wb, fmt=fmt, scale="e4m3_mean")
+    w = gpu_quant(lib, Wb, fmt, "e4m3_mean")
+    assert w.c1.numel() == 2 * ((N * K // 64 + 255) // 256)
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, N, K, fmt=fmt, scale="e4m3_mean"))
+
+
+def test_mean_scales_every_significand_pair(lib):
+    """The significand-pair matrix (group sums stay finite: absmax values up
+    to about 1e30 only), where scales of very different size share groups
+    and the residuals take both signs."""
+    Wb = mantissa_pair_matrix()
+    cmax = O.bf16_bits_to_f32(Wb[:, 0])
+    Wb = Wb[cmax < 1e30]
+    Wb = Wb[: (Wb.shape[0] // 4) * 4]
+    ref = O.quantize(Wb, scale="e4m3_mean")
+    assert np.any(ref[1] & 0x80) and np.any((ref[1] & 0x80) == 0)      # residuals of both signs
+    w = gpu_quant(lib, Wb, "nf4", "e4m3_mean")
+    assert_quant_equal(w, ref)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, *Wb.shape, scale="e4m3_mean"))
+
+
+def test_mean_scales_equal_blocks_reconstruct(lib):
+    """A group of 256 blocks with the same absmax: c1 = 0, all c2 = 0 and the
+    decoded scale is the mean, i.e. exactly the absmax."""
+    blk = np.zeros((256, 64), np.float32)
+    blk[:, 0] = 0.0234375
+    blk[:, 9] = -0.01
+    Wb = O.f32_to_bf16_bits(blk).reshape(64, 256)
+    ref = O.quantize(Wb, scale="e4m3_mean")
+    w = gpu_quant(lib, Wb, "nf4", "e4m3_mean")
+    assert_quant_equal(w, ref)
+    assert ref[2][0] == 0 and np.all(ref[1] == 0)
+    assert np.array_equal(bits(lib.dequant(w)), O.dequant(*ref, 64, 256, scale="e4m3_mean"))
+
+
 def test_quantize_sharded_single_rank_equals_quantize(lib):
     """The sharded quantiser's per-rank step (the library quantiser on a flat
     [1, len] view of a run of whole 16384-weight groups) without a process
