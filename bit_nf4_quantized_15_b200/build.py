@@ -18,8 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqlora_nf4.so")
-SOURCES = ["api.cu", "engine.cu", "engine_pair.cu", "gemv.cu", "quant.cu", "adapters.cu", "noalloc.cu",
-           "nf4_tables.cpp"]
+SOURCES = ["api.cu", "engine.cu", "engine_pair.cu", "gemv.cu", "gemv_bwd.cu", "quant.cu", "adapters.cu",
+           "noalloc.cu", "nf4_tables.cpp"]
 HEADERS = ["common.cuh", "engine_util.cuh", "internal.h"]
 
 

@@ -194,7 +194,8 @@ bool valid_rank(int r) { return r >= 8 && r <= 128 && r % 8 == 0; }
 struct WsLayout {
   size_t ofs_sdT, ofs_partial, total;
   GemmPlan t_fwd, y_fwd, dt, dx, dl1, dl2;
-  GemvPlan gemv;  // M <= kGemvMaxM only
+  GemvPlan gemv;    // M <= kGemvMaxM only
+  GemvTPlan gemvt;  // M <= kGemvMaxM only
 };
 
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
@@ -212,10 +213,13 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t part = 0;
   for (const GemmPlan* p : {&w.t_fwd, &w.y_fwd, &w.dt, &w.dx, &w.dl1, &w.dl2})
     part = p->partial_bytes > part ? p->partial_bytes : part;
-  if (M <= kGemvMaxM) {  // few-token forward: stream-K partials + T slices
+  if (M <= kGemvMaxM) {  // few tokens: stream-K partials + T / dT slices (+ arrival counters)
     w.gemv = plan_gemv(M, N, K, sms);
     const size_t g = align256(w.gemv.part_bytes) + align256(w.gemv.tp_bytes) + w.gemv.stw_bytes;
     part = g > part ? g : part;
+    w.gemvt = plan_gemv_t(M, N, K, sms);
+    const size_t gt = align256(w.gemvt.part_bytes) + align256(w.gemvt.tp_bytes) + w.gemvt.cnt_bytes;
+    part = gt > part ? gt : part;
   }
   w.total = w.ofs_partial + align256(part);
   return w;
@@ -524,6 +528,51 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const flo
   uint16_t* sT = reinterpret_cast<uint16_t*>(wsb);
   uint16_t* sdT = reinterpret_cast<uint16_t*>(wsb + lay.ofs_sdT);
   float* partial = reinterpret_cast<float*>(wsb + lay.ofs_partial);
+
+  if (M <= kGemvMaxM) {
+    // Few tokens: weight-streaming backward (dT and dL2 over N slices, then
+    // dX and dL1 by stream-K over the weight).
+    const GemvTPlan& gp = lay.gemvt;
+    GemvTArgs ga;
+    std::memset(&ga, 0, sizeof(ga));
+    if (make_map(&ga.tmCodes, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+        make_map(&ga.tmDY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)N, (uint64_t)M, 64, 16,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+      return QLORA_ERR_CUDA;
+    ga.c2 = w->c2;
+    ga.c1 = w->c1;
+    ga.c2_e5m2 = w->scale_codec == QLORA_SCALE_E5M2;
+    ga.c1_mean = w->scale_codec == QLORA_SCALE_E4M3_MEAN;
+    ga.N = N;
+    ga.K = K;
+    ga.M = (int)M;
+    ga.r = r;
+    ga.kbt = gp.kbt;
+    ga.n_tiles = gp.n_tiles;
+    ga.maxc = gp.maxc;
+    ga.t_slices = gp.t_slices;
+    ga.units = gp.units;
+    ga.s = s;
+    uint8_t* g0 = wsb + lay.ofs_partial;
+    ga.part = reinterpret_cast<float*>(g0);
+    ga.tp = reinterpret_cast<float*>(g0 + align256(gp.part_bytes));
+    ga.cnt = reinterpret_cast<int*>(g0 + align256(gp.part_bytes) + align256(gp.tp_bytes));
+    ga.L1 = L1;
+    ga.X = X;
+    ga.dX = dX;
+    ga.dL1 = dL1;
+    ga.status = status_dev;
+    const Nf4Tables& tb = code_tables(w->format);
+    for (int i = 0; i < 16; ++i) ga.q[i] = tb.q[i];
+    cudaEvent_t e0 = g_ev_start, e1 = g_ev_end;
+    g_ev_start = g_ev_end = nullptr;
+    g_stall_ns = 0;
+    if (e0 && cudaEventRecord(e0, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_gemv_t(ga, gp, dY, L2, T_saved, dL2, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (e1 && cudaEventRecord(e1, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
 
   // (0) s.T in bf16, the operand of dL2.
   if (dL2 && launch_scale_to_bf16(T_saved, M * r, s, sT, st) != cudaSuccess) return QLORA_ERR_CUDA;

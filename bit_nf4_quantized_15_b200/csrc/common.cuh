@@ -48,11 +48,16 @@ QDEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-QDEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Non-blocking test of a phase (test_wait, with acquire semantics).  The
+// waits below poll with it rather than with try_wait: try_wait may suspend
+// the thread, and a suspended waiter was measured to resume about 0.5 us
+// after the phase completed, which put a floor under every pipeline stage
+// (one TMA box per 0.5 us per waiting producer).
+QDEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -62,16 +67,16 @@ QDEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete.  Bounded: returns
 // false (after flagging the CTA and the caller's status) on timeout or when
-// another role of the CTA has already aborted.  Plain polling: a suspended
-// wait (try_wait with a time hint) was measured to wake up late.
+// another role of the CTA has already aborted.  Plain polling with test_wait
+// (see mbar_test_wait).
 // `limit_ns` is the bound (QNF4_WAIT_NS unless a launch asks for less).
 QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
                     uint64_t limit_ns = QNF4_WAIT_NS) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  if (mbar_test_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (mbar_test_wait(a, parity)) return true;
     if ((i & 63) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
@@ -89,11 +94,11 @@ QDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, in
 QDEV bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
                             uint32_t sleep_ns, uint64_t limit_ns = QNF4_WAIT_NS) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  if (mbar_test_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (;;) {
     __nanosleep(sleep_ns);
-    if (mbar_try_wait(a, parity)) return true;
+    if (mbar_test_wait(a, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
@@ -107,7 +112,7 @@ QDEV bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort_
 QDEV void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t ns) {
   const uint32_t a = smem_u32(bar);
   const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(a, parity)) {
+  while (!mbar_test_wait(a, parity)) {
     if (globaltimer() - t0 > ns) return;
   }
 }

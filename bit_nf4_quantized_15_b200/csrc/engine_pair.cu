@@ -92,11 +92,11 @@ QDEV void cluster_sync_all() {
 QDEV void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-QDEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+QDEV bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -106,10 +106,10 @@ QDEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
 // Bounded wait with cluster-scope acquire (arrivals from the peer CTA).
 QDEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cluster(a, parity)) return true;
+  if (mbar_test_wait_cluster(a, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cluster(a, parity)) return true;
+    if (mbar_test_wait_cluster(a, parity)) return true;
     if ((i & 63) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > QNF4_WAIT_NS) {

@@ -146,7 +146,7 @@ QDEV bool warp_wait_g(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
   int ok = 1;
   if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
   ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  if (ok) mbar_try_wait(smem_u32(bar), parity);
+  if (ok) mbar_test_wait(smem_u32(bar), parity);
   return ok != 0;
 }
 

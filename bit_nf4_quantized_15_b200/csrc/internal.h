@@ -156,6 +156,49 @@ GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& p, const uint16_t* X, const uint16_t* L1,
                         const uint16_t* L2, uint16_t* Y, cudaStream_t st);
 
+// ------------------------------------------------- small-M backward (GEMV)
+// Backward for M <= kGemvMaxM tokens with the weight streamed once:
+//   (1) lora_bwd_n_kernel: over N slices, dL2 = s.T^T.dY and the slices'
+//       partials of dT = dY.L2^T; zeroes the k-range arrival counters;
+//   (2) nf4_gemv_t_kernel: dX = dY.W^ by stream-K over units (128-row tile
+//       of W, 256-wide k range) ordered by k range; the last worker of a k
+//       range adds s.dT.L1^T, rounds dX and forms dL1 = s.X^T.dT there.
+struct GemvTPlan {
+  int n_tiles, kbt, k_ranges;  // 128-row tiles of W, 64-wide k blocks, 256-wide k ranges
+  int64_t units;               // n_tiles * k_ranges
+  int grid, workers, maxc;     // CTAs, stream-K workers (3 per CTA), max workers per k range
+  int slice, t_slices;         // dT slices over N
+  size_t part_bytes;           // [k_ranges][maxc][16][256] fp32
+  size_t tp_bytes;             // [t_slices][16][128] fp32
+  size_t cnt_bytes;            // [k_ranges] int
+};
+
+struct GemvTArgs {
+  CUtensorMap tmCodes;  // uint8 [N][K/2], box 128 x 128, 128-byte swizzle
+  CUtensorMap tmDY;     // bf16 [M][N], box 64 x 16, 128-byte swizzle
+  const uint8_t* c2;
+  int c2_e5m2, c1_mean;
+  const float* c1;
+  int64_t N, K;
+  int M, r, kbt, n_tiles, maxc, t_slices;
+  int64_t units;
+  float s;
+  float* part;
+  const float* tp;
+  int* cnt;
+  const uint16_t* L1;
+  const uint16_t* X;
+  uint16_t* dX;   // may be null
+  float* dL1;     // may be null
+  int* status;
+  uint32_t smem_bytes;
+  float q[16];
+};
+
+GemvTPlan plan_gemv_t(int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv_t(const GemvTArgs& a, const GemvTPlan& p, const uint16_t* dY, const uint16_t* L2,
+                          const float* T, float* dL2, cudaStream_t st);
+
 // --------------------------------------------------------- quantise kernels
 cudaError_t launch_quantize(const uint16_t* W, int64_t n_weights, uint8_t* codes, uint8_t* c2, float* c1,
                             int* status, int format, int scale_codec, cudaStream_t st);
