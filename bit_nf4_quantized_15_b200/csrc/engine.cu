@@ -4,7 +4,8 @@
 //
 // One CTA computes a 128 x BN output tile with cta_group::1 UMMA (M = 128).
 // The reduction runs in 64-wide blocks through a 4-stage shared-memory ring:
-//   * warp 0, one lane: TMA producer (B tiles, A tiles or NF4 code tiles);
+//   * warp 0, one lane per ring stage: TMA producers (B tiles, A tiles or
+//     NF4 code tiles);
 //   * warp 1, one lane: UMMA issuer, 4 x (128 x BN x 16) MMAs per stage,
 //     tcgen05.commit frees the stage;
 //   * warps 2..5 (128 threads): when A is the NF4 weight, they turn the code
@@ -122,8 +123,12 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && !args.stall) {
-      for (int it = 0; it < n_iters; ++it) {
+    // One lane per ring stage: a thread keeps about one large TMA box in
+    // flight at a time (measured on B200: ~0.55 us per box per issuing
+    // thread whatever the ring depth, while boxes from different threads
+    // overlap), so each stage has its own issuing lane.
+    if (lane < kStages && !args.stall) {
+      for (int it = lane; it < n_iters; it += kStages) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status, lim)) break;

@@ -247,13 +247,15 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
   __syncthreads();
 
   if (warp == 0) {
-    // ----------------------------------------------- producers (lanes 0..2)
-    if (lane < kWG) {
-      const int g = lane, wk = c * kWG + g;
+    // ------------------------------------ producers: one lane per ring stage
+    // (lane 2g + j fills stage j of worker g; a thread keeps about one
+    // large TMA box in flight at a time)
+    if (lane < kWG * kWS) {
+      const int g = lane / kWS, wk = c * kWG + g;
       const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
       const int nu = (int)(u1 - u0);
       int issued = 0;
-      for (int i = 0; i < nu; ++i) {
+      for (int i = lane % kWS; i < nu; i += kWS) {
         const int j = i % kWS;
         if (!mbar_wait_backoff(bar_empty(S, g, j), ((uint32_t)(i / kWS) & 1u) ^ 1u, S.abort_flag, args.status, 128))
           break;
@@ -267,9 +269,9 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
         tma_load_3d(sp + kCodeBytes, &args.tmX, bar_full(S, g, j), 0, 0, un * kUnitKB);
         issued = i + 1;
       }
-      if (*S.abort_flag) {  // let the loads already issued land before exit
-        for (int i = issued - kWS > 0 ? issued - kWS : 0; i < issued; ++i)
-          mbar_wait_drain(bar_full(S, g, i % kWS), (uint32_t)(i / kWS) & 1u, 10000000ull);
+      if (*S.abort_flag && issued > 0) {  // let this lane's last load land before exit
+        const int i = issued - 1;
+        mbar_wait_drain(bar_full(S, g, i % kWS), (uint32_t)(i / kWS) & 1u, 10000000ull);
       }
     }
   } else if (warp == kWarpT) {
@@ -515,7 +517,9 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
   for (int q = 0; q < 32; ++q)
     l2v[q] = (valid && q < rq) ? bf16_bits_to_float(__ldg(L2 + (int64_t)(j0 + q) * N + n)) : 0.0f;
   grid_dep_wait();
-  for (int idx = t; idx < M * 128; idx += 128) sT[idx] = sTw[idx];
+#pragma unroll 4
+  for (int idx = t * 4; idx < M * 128; idx += 128 * 4)  // 16-byte pieces, several in flight
+    *reinterpret_cast<float4*>(sT + idx) = __ldcg(reinterpret_cast<const float4*>(sTw + idx));
   const int c_lo = worker_of((int64_t)rt * upr, U, W);
   const int cnt = min(worker_of((int64_t)(rt + 1) * upr - 1, U, W) - c_lo + 1, maxc);
   float acc[MB];

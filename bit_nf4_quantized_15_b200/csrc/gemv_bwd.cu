@@ -179,9 +179,16 @@ __global__ void __launch_bounds__(256) lora_bwd_n_kernel(const uint16_t* __restr
       *reinterpret_cast<uint4*>(sY + m * kBChunk + c * 8) =
           __ldg(reinterpret_cast<const uint4*>(dY + (int64_t)m * N + n0) + c);
     }
-    for (int i = t; i < r * cw; i += 256) {               // L2 [j][n] -> sL [n][j]
-      const int j = i / cw, nn = i % cw;
-      sL[nn * r + j] = __ldg(L2 + (int64_t)j * N + n0 + nn);
+#pragma unroll 4
+    for (int i = t; i < r * (cw / 8); i += 256) {         // L2 [j][n] -> sL [n][j], 16-byte loads
+      const int j = i / (cw / 8), c = i % (cw / 8);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(L2 + (int64_t)j * N + n0) + c);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sL[(c * 8 + 2 * e) * r + j] = (uint16_t)(w4[e] & 0xFFFFu);
+        sL[(c * 8 + 2 * e + 1) * r + j] = (uint16_t)(w4[e] >> 16);
+      }
     }
     __syncthreads();
     if (dL2) {                                            // dL2[j][n] = s . sum_m T[m][j] dY[m][n]
@@ -253,13 +260,13 @@ __global__ void __launch_bounds__(kTThreads, 1) nf4_gemv_t_kernel(const __grid_c
   __syncthreads();
 
   if (warp == 0) {
-    // ----------------------------------------------- producers (lanes 0..2)
-    if (lane < kTG) {
-      const int g = lane, wk = c * kTG + g;
+    // ------------------------------------ producers: one lane per ring stage
+    if (lane < kTG * kTS) {
+      const int g = lane / kTS, wk = c * kTG + g;
       const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
       const int nu = (int)(u1 - u0);
       int issued = 0;
-      for (int i = 0; i < nu; ++i) {
+      for (int i = lane % kTS; i < nu; i += kTS) {
         const int j = i % kTS;
         if (!mbar_wait_backoff(tempty(S, g, j), ((uint32_t)(i / kTS) & 1u) ^ 1u, S.abort_flag, args.status, 64))
           break;
@@ -272,9 +279,9 @@ __global__ void __launch_bounds__(kTThreads, 1) nf4_gemv_t_kernel(const __grid_c
         tma_load_2d(sp + kTCode + 2048, &args.tmDY, tfull(S, g, j), nt * 128 + 64, 0);
         issued = i + 1;
       }
-      if (*S.abort_flag) {
-        for (int i = issued - kTS > 0 ? issued - kTS : 0; i < issued; ++i)
-          mbar_wait_drain(tfull(S, g, i % kTS), (uint32_t)(i / kTS) & 1u, 10000000ull);
+      if (*S.abort_flag && issued > 0) {
+        const int i = issued - 1;
+        mbar_wait_drain(tfull(S, g, i % kTS), (uint32_t)(i / kTS) & 1u, 10000000ull);
       }
     }
     return;  // no barrier below involves warp 0
@@ -411,42 +418,103 @@ __global__ void __launch_bounds__(kTThreads, 1) nf4_gemv_t_kernel(const __grid_c
     if (!S.fix_flag[g]) continue;
     __threadfence();
     t_dep_wait();  // the dT slice partials
-    // dT = sum of the slice partials (slice order) into this worker's region
+    // dT = sum of the slice partials (slice order) into this worker's region,
+    // eight loads in flight per element
     const uint32_t fix = S.fix + (uint32_t)(g * kTFix);
     for (int e = tw; e < args.M * args.r; e += 32 * kTW) {
       const int m = e / args.r, jj = e % args.r;
+      const float* src = args.tp + (int64_t)m * 128 + jj;
       float a = 0.0f;
-      for (int p = 0; p < args.t_slices; ++p) a += __ldcg(args.tp + ((int64_t)p * 16 + m) * 128 + jj);
+      for (int p0 = 0; p0 < args.t_slices; p0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = p0 + q < args.t_slices ? __ldcg(src + (int64_t)(p0 + q) * 16 * 128) : 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (p0 + q < args.t_slices) a += v[q];
+      }
       sts_f32(fix + (uint32_t)((m * 128 + jj) * 4), a);
     }
     named_sync(1 + g, 32 * kTW);
     const int c_lo = t_worker_of((int64_t)kr * ntl, U, W);
     const int cnt_c = min(t_worker_of((int64_t)kr * ntl + ntl - 1, U, W) - c_lo + 1, args.maxc);
-    for (int kk = 0; kk < 2; ++kk) {
-      const int kl = 2 * tw + kk;
-      const int64_t k = (int64_t)kr * 256 + kl;
-      if (k >= args.K) continue;
+    const int kl = 2 * tw;  // this thread: columns k, k + 1 of the k range
+    const int64_t k = (int64_t)kr * 256 + kl;
+    if (k < args.K) {       // K % 64 == 0: k + 1 < K as well
       if (args.dX) {
-        for (int m = 0; m < args.M; ++m) {
-          float a = 0.0f;
-          for (int jc = 0; jc < cnt_c; ++jc) a += __ldcg(args.part + (((int64_t)kr * args.maxc + jc) * 16 + m) * 256 + kl);
-          float l = 0.0f;
-          for (int jj = 0; jj < args.r; ++jj)
-            l = __fmaf_rn(lds_f32(fix + (uint32_t)((m * 128 + jj) * 4)), bf16_bits_to_float(__ldg(args.L1 + k * args.r + jj)), l);
-          reinterpret_cast<__nv_bfloat16*>(args.dX)[(int64_t)m * args.K + k] =
-              __float2bfloat16_rn(__fmaf_rn(args.s, l, a));
+        // the segment partials of every token, in worker order, two workers at a time
+        float2 acc2[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc2[m] = make_float2(0.0f, 0.0f);
+        const float* pbase = args.part + (int64_t)kr * args.maxc * (16 * 256) + kl;
+        for (int jc = 0; jc < cnt_c; jc += 2) {
+          float2 v0[16], v1[16];
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            v0[m] = m < args.M ? __ldcg(reinterpret_cast<const float2*>(pbase + ((int64_t)jc * 16 + m) * 256))
+                               : make_float2(0.0f, 0.0f);
+            v1[m] = (m < args.M && jc + 1 < cnt_c)
+                        ? __ldcg(reinterpret_cast<const float2*>(pbase + ((int64_t)(jc + 1) * 16 + m) * 256))
+                        : make_float2(0.0f, 0.0f);
+          }
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            acc2[m].x += v0[m].x;
+            acc2[m].y += v0[m].y;
+            if (jc + 1 < cnt_c) {
+              acc2[m].x += v1[m].x;
+              acc2[m].y += v1[m].y;
+            }
+          }
         }
+        // + s . dT . L1^T for the two columns, L1 rows read eight adapter columns at a time
+        float2 l2[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) l2[m] = make_float2(0.0f, 0.0f);
+        for (int j0 = 0; j0 < args.r; j0 += 8) {
+          const uint4 la = __ldg(reinterpret_cast<const uint4*>(args.L1 + k * args.r + j0));
+          const uint4 lb = __ldg(reinterpret_cast<const uint4*>(args.L1 + (k + 1) * args.r + j0));
+          const uint32_t wa[4] = {la.x, la.y, la.z, la.w}, wb[4] = {lb.x, lb.y, lb.z, lb.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float fa = bf16_bits_to_float((wa[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+            const float fb = bf16_bits_to_float((wb[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              if (m < args.M) {
+                const float tv = lds_f32(fix + (uint32_t)((m * 128 + j0 + q) * 4));
+                l2[m].x = __fmaf_rn(tv, fa, l2[m].x);
+                l2[m].y = __fmaf_rn(tv, fb, l2[m].y);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          if (m < args.M)
+            *reinterpret_cast<uint32_t*>(args.dX + (int64_t)m * args.K + k) =
+                pack_bf16x2(__fmaf_rn(args.s, l2[m].x, acc2[m].x), __fmaf_rn(args.s, l2[m].y, acc2[m].y));
       }
       if (args.dL1) {
-        float xm[16];
+        float xa[16], xb[16];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) xm[m] = m < args.M ? bf16_bits_to_float(__ldg(args.X + (int64_t)m * args.K + k)) : 0.0f;
+        for (int m = 0; m < 16; ++m) {
+          const uint32_t xv = m < args.M ? __ldg(reinterpret_cast<const uint32_t*>(args.X + (int64_t)m * args.K + k)) : 0u;
+          xa[m] = bf16_bits_to_float(xv & 0xFFFFu);
+          xb[m] = bf16_bits_to_float(xv >> 16);
+        }
         for (int jj = 0; jj < args.r; ++jj) {
-          float a = 0.0f;
+          float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-          for (int m = 0; m < 16; ++m)
-            if (m < args.M) a = __fmaf_rn(xm[m], lds_f32(fix + (uint32_t)((m * 128 + jj) * 4)), a);
-          args.dL1[k * args.r + jj] = __fmul_rn(args.s, a);
+          for (int m = 0; m < 16; ++m) {
+            if (m < args.M) {
+              const float tv = lds_f32(fix + (uint32_t)((m * 128 + jj) * 4));
+              a0 = __fmaf_rn(xa[m], tv, a0);
+              a1 = __fmaf_rn(xb[m], tv, a1);
+            }
+          }
+          args.dL1[k * args.r + jj] = __fmul_rn(args.s, a0);
+          args.dL1[(k + 1) * args.r + jj] = __fmul_rn(args.s, a1);
         }
       }
     }
