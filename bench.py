@@ -50,8 +50,10 @@ METRIC = ("fused QLoRA linear fwd+bwd TFLOP/s and % of roofline; "
           "NF4 (de)quant GB/s vs HBM peak")
 WORKLOAD = "llama65b_block"
 # DRAM bytes (read + write) per fused dequant-GEMM launch of the headline
-# step, from an ncu capture of the current kernels; None until one exists.
-FUSED_TRAFFIC_BYTES = None
+# step: the mean over its 14 fused launches (Y and dX of the 7 linears) of
+# dram__bytes_read.sum + dram__bytes_write.sum, one single-pass ncu capture
+# of `bench.py --no-extras --no-cpu-baseline --steps 1 --warmup 1`.
+FUSED_TRAFFIC_BYTES = 923.3e6
 RT_WORKLOAD = ("bulk NF4 round trip of 2^31 bf16 weights (4 GiB): half N(0, 0.02), half Student-t(3) x 0.02 "
                "with 0.1% outliers x50; one launch per direction")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -308,6 +310,10 @@ class BlockStep:
         self.flops = sum(linear_flops(M, l.N, l.K, r) for l in wl.linears)
         self.y_flops = sum(fwd_gemm_flops(M, l.N, l.K, r) for l in wl.linears)
         self.dx_flops = sum(dx_gemm_flops(M, l.N, l.K, r) for l in wl.linears)
+        # bytes the two fused launches of a linear must move: NF4 weight, the
+        # activation in (X or dY), the output (Y or dX), adapters and s.T / s.dT
+        self.fused_bytes = sum(2 * nf4_bytes(l.N, l.K) + 2 * 2 * M * (l.K + l.N) + 2 * 2 * r * (l.K + l.N)
+                               + 2 * 2 * M * r for l in wl.linears)
 
     def step(self, events=None, exchange=False):
         q, s = self.q, self.wl.s
@@ -634,6 +640,7 @@ def run_ours(args):
         "dx": {"achieved": dx_ach, "frac": dx_ach / peak, "ms_per_step": res["dx_ms"],
                "flops_per_step": blk.dx_flops},
         "flops_note": "algorithmic: 2 M K N + 2 M r (N or K) per launch; the dequantisation is not counted",
+        "algorithmic_bytes_per_launch": blk.fused_bytes / (2 * n_lin),
     }
 
     line_extra = {}

@@ -26,6 +26,7 @@ namespace qnf4 {
 namespace {
 
 constexpr int kGroupWarps = 4;  // a dequant group: 4 warps, one per TMEM lane quarter
+constexpr int kRasterGroup = 4;  // column tiles per raster group (see the kernel's tile mapping)
 
 // Ring shape per A source.  The forward keeps its dequantised A tile in
 // TMEM, so its stages hold only B and the codes (36 KB) and six of them fit:
@@ -82,7 +83,22 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row0 = blockIdx.x * 128, col0 = blockIdx.y * BN, z = blockIdx.z;
+  // Grouped raster over the linear block index: consecutive CTAs take up to
+  // kRasterGroup column tiles (tokens) of one row tile (weight), then the
+  // next row tile.  The CTAs resident at a time then share a few activation
+  // tiles (kept in L2) and each weight tile's codes are read from HBM once
+  // per group of column tiles instead of once per column tile.
+  int row_tile, col_tile;
+  {
+    const int m_tiles = (args.rows + 127) / 128, n_tiles = (args.cols + BN - 1) / BN;
+    const int id = blockIdx.x;
+    const int per_group = kRasterGroup * m_tiles;
+    const int gid = id / per_group, local = id % per_group;
+    const int gsize = min(kRasterGroup, n_tiles - gid * kRasterGroup);
+    col_tile = gid * kRasterGroup + local % gsize;
+    row_tile = local / gsize;
+  }
+  const int row0 = row_tile * 128, col0 = col_tile * BN, z = blockIdx.z;
   const int kb_lo = (int)((int64_t)z * args.kb_main / args.splits);
   const int kb_hi = (int)((int64_t)(z + 1) * args.kb_main / args.splits);
   const int my_kb = kb_hi - kb_lo;
@@ -400,7 +416,7 @@ cudaError_t launch_t(const EngineArgs& a, const GemmPlan& p, cudaStream_t st) {
   auto kern = umma_engine_kernel<BN, AMODE>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
   if (err != cudaSuccess) return err;
-  dim3 grid(p.m_tiles, p.n_tiles, p.splits);
+  dim3 grid(p.m_tiles * p.n_tiles, 1, p.splits);
   kern<<<grid, Ring<AMODE>::THREADS, L::TOTAL, st>>>(a);
   count_launches(1);
   return cudaGetLastError();
