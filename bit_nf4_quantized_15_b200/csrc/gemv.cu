@@ -59,7 +59,7 @@ constexpr int kCodeBytes = 16384;          // 128 rows x 128 bytes (256 codes)
 constexpr int kXBytes = 8192;              // 16 tokens x 256 bf16: one 3-D box of 4 x (16 x 64)
 constexpr int kStageBytes = kCodeBytes + kXBytes;
 // A worker's warps each own kRG 16-row groups of the 128-row tile.
-constexpr int kRG = 2;
+constexpr int kRG = 1;
 constexpr int kWW = 8 / kRG;                  // warps per worker
 // Warps: 0 producers, 1 .. kWW*kWG workers, last: T reduction.
 constexpr int kWarpT = 1 + kWW * kWG;
@@ -324,7 +324,6 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
     for (int i = 0; i < nu; ++i) {
       const int64_t u = u0 + i;
       const int rt = (int)(u / upr), un = (int)(u % upr);
-      const int nkb = min(kUnitKB, args.kbt - un * kUnitKB);
       const bool seg_end = i == nu - 1 || un == upr - 1;
       float chs[2 * kRG][kUnitKB];  // c^ of this unit's blocks, per thread row
 #pragma unroll
@@ -342,7 +341,9 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
         const uint32_t st = stage_addr(S, kWS * g + j);
 #pragma unroll
         for (int q = 0; q < kUnitKB; ++q) {
-          if (q >= nkb) break;
+          // (blocks beyond K in the last unit of a row: zero codes and X from
+          // the TMA fill, zero scales, so they add nothing; no branch keeps
+          // the four blocks unrolled and interleaved)
           // X fragments of the four k-steps: token n = 8t + gr, k = 16cq + 4s .. +3
           uint2 xb[NT][4];
           const uint32_t xt = st + kCodeBytes + (uint32_t)q * 2048;
