@@ -4,8 +4,8 @@
 //
 // One CTA computes a 128 x BN output tile with cta_group::1 UMMA (M = 128).
 // The reduction runs in 64-wide blocks through a 4-stage shared-memory ring:
-//   * warp 0, one lane per ring stage: TMA producers (B tiles, A tiles or
-//     NF4 code tiles);
+//   * warp 0, one lane: TMA producer (B tiles, A tiles or NF4 code tiles),
+//     stages in order;
 //   * warp 1, one lane: UMMA issuer, 4 x (128 x BN x 16) MMAs per stage,
 //     tcgen05.commit frees the stage;
 //   * warps 2..5 (128 threads): when A is the NF4 weight, they turn the code
@@ -139,12 +139,12 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // One lane per ring stage: a thread keeps about one large TMA box in
-    // flight at a time (measured on B200: ~0.55 us per box per issuing
-    // thread whatever the ring depth, while boxes from different threads
-    // overlap), so each stage has its own issuing lane.
-    if (lane < kStages && !args.stall) {
-      for (int it = lane; it < n_iters; it += kStages) {
+    // One thread issues every stage in order.  (Spreading the stages over
+    // several lanes of this warp, each spinning on its own barrier, was
+    // measured slower: divergent spinning lanes of one warp take turns, so a
+    // lane whose stage is free can wait behind another's spin loop.)
+    if (lane == 0 && !args.stall) {
+      for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.status, lim)) break;
@@ -189,8 +189,13 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         const bool ext = it >= my_kb;
-        bool ok = mbar_wait(full + s, ph, abort_flag, args.status, lim);
-        if (ok && AMODE != A_TMA && !ext) ok = mbar_wait(afull + s, ph, abort_flag, args.status, lim);
+        // A dequantised stage is waited on through afull alone: its group
+        // arrives there only after it has seen the stage's TMA bytes land
+        // (full, acquire), so the B tile is complete too, and one barrier
+        // read per stage is saved on this thread's critical path (a
+        // shared-memory access costs it ~0.2 us while the tensor core and
+        // the TMA stream through shared memory).
+        const bool ok = mbar_wait(AMODE != A_TMA && !ext ? afull + s : full + s, ph, abort_flag, args.status, lim);
         if (!ok) break;
         tc_fence_after();
         const uint8_t* sa = smem + s * L::STAGE;
