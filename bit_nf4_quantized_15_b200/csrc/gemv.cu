@@ -245,6 +245,9 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(S.tab + (uint32_t)(e * 256 + l * 4)), "r"(v) : "memory");
   }
   __syncthreads();
+  // The finish kernel may be launched now: it reads this kernel's results
+  // only after griddepcontrol.wait, and its launch latency overlaps the GEMV.
+  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------ producers: one lane per ring stage
@@ -423,8 +426,6 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
     }
   }
 
-  __syncthreads();
-  grid_dep_launch();
 }
 
 // T partials: Tp[p][m][j] = sum over the k of slice p of X[m,k] L1[k,j], fp32,
@@ -495,55 +496,55 @@ __global__ void __launch_bounds__(256) lora_t_partial_kernel(const uint16_t* __r
   }
 }
 
-// Y for 32 weight rows per CTA (128 threads), tokens m < MB (M <= MB).  Warp
-// w sums the row tile's partials of contributors j = w, w + 4, ... and the
-// LoRA products of adapter columns [w*r/4, (w+1)*r/4); the four warps' sums
-// are then added in warp order.
+// Y for 32 weight rows per CTA (512 threads), tokens m < MB (M <= MB).
+// Warp w sums the row tile's partials of contributors j = w, w + 16, ...
+// (all of a warp's loads in flight together) and the LoRA products of
+// adapter columns j = w, w + 16, ...; the sixteen warps' sums are then added
+// in warp order (fixed, so the result is repeatable).
+constexpr int kFinWarps = 16;
 template <int MB>
-__global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restrict__ part,
-                                                          const float* __restrict__ sTw,
-                                                          const uint16_t* __restrict__ L2, int M, int64_t N, int r,
-                                                          int upr, int64_t U, int W, int maxc,
-                                                          uint16_t* __restrict__ Y) {
+__global__ void __launch_bounds__(32 * kFinWarps) gemv_finish_kernel(const float* __restrict__ part,
+                                                                    const float* __restrict__ sTw,
+                                                                    const uint16_t* __restrict__ L2, int M,
+                                                                    int64_t N, int r, int upr, int64_t U, int W,
+                                                                    int maxc, uint16_t* __restrict__ Y) {
   __shared__ __align__(16) float sT[16 * 128];
-  __shared__ float red[4][MB][32];
+  __shared__ float red[kFinWarps][MB][32];
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int64_t n0 = (int64_t)blockIdx.x * 32, n = n0 + lane;
   const int rt = (int)(n0 / 128), rl = (int)(n % 128);
   const bool valid = n < N;
-  const int rq = r / 4, j0 = w * rq;  // this warp's adapter columns (r % 8 == 0, so rq is even)
-  // L2 first: it does not depend on the previous kernels
-  float l2v[32];
+  // L2 first: it does not depend on the previous kernels (r <= 128: at most 8 columns per warp)
+  float l2v[8];
 #pragma unroll
-  for (int q = 0; q < 32; ++q)
-    l2v[q] = (valid && q < rq) ? bf16_bits_to_float(__ldg(L2 + (int64_t)(j0 + q) * N + n)) : 0.0f;
+  for (int q = 0; q < 8; ++q) {
+    const int j = w + kFinWarps * q;
+    l2v[q] = (valid && j < r) ? bf16_bits_to_float(__ldg(L2 + (int64_t)j * N + n)) : 0.0f;
+  }
   grid_dep_wait();
-#pragma unroll 4
-  for (int idx = t * 4; idx < M * 128; idx += 128 * 4)  // 16-byte pieces, several in flight
+  for (int idx = t * 4; idx < M * 128; idx += 32 * kFinWarps * 4)  // 16-byte pieces
     *reinterpret_cast<float4*>(sT + idx) = __ldcg(reinterpret_cast<const float4*>(sTw + idx));
   const int c_lo = worker_of((int64_t)rt * upr, U, W);
   const int cnt = min(worker_of((int64_t)(rt + 1) * upr - 1, U, W) - c_lo + 1, maxc);
   float acc[MB];
 #pragma unroll
   for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
-  for (int j = w; j < cnt; j += 4) {
+  for (int j = w; j < cnt; j += kFinWarps) {
     const float* src = part + ((int64_t)rt * maxc + j) * (16 * 128) + rl;
+    float v[MB];
 #pragma unroll
-    for (int m = 0; m < MB; ++m)
-      if (m < M) acc[m] += src[m * 128];
+    for (int m = 0; m < MB; ++m) v[m] = m < M ? __ldcg(src + m * 128) : 0.0f;
+#pragma unroll
+    for (int m = 0; m < MB; ++m) acc[m] += v[m];
   }
   __syncthreads();
 #pragma unroll
-  for (int q2 = 0; q2 < 16; ++q2) {
-    if (q2 * 2 < rq) {  // j0 + 2 q2 is even: 8-byte aligned pairs of s.T
+  for (int q = 0; q < 8; ++q) {
+    const int j = w + kFinWarps * q;
+    if (j < r) {
 #pragma unroll
-      for (int m = 0; m < MB; ++m) {
-        if (m < M) {
-          const float2 s2 = *reinterpret_cast<const float2*>(sT + m * 128 + j0 + q2 * 2);
-          acc[m] = __fmaf_rn(s2.x, l2v[q2 * 2 + 0], acc[m]);
-          acc[m] = __fmaf_rn(s2.y, l2v[q2 * 2 + 1], acc[m]);
-        }
-      }
+      for (int m = 0; m < MB; ++m)
+        if (m < M) acc[m] = __fmaf_rn(sT[m * 128 + j], l2v[q], acc[m]);
     }
   }
 #pragma unroll
@@ -553,7 +554,9 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
 #pragma unroll
     for (int m = 0; m < MB; ++m)
       if (m < M) {
-        const float y = ((red[0][m][lane] + red[1][m][lane]) + red[2][m][lane]) + red[3][m][lane];
+        float y = red[0][m][lane];
+#pragma unroll
+        for (int q = 1; q < kFinWarps; ++q) y += red[q][m][lane];
         reinterpret_cast<__nv_bfloat16*>(Y)[(int64_t)m * N + n] = __float2bfloat16_rn(y);
       }
   }
@@ -592,6 +595,15 @@ GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int num_sms) {
   const int64_t min_run = p.units / p.workers;  // 0 when some workers get nothing
   p.maxc = min_run > 0 ? (int)((p.upr + min_run - 1) / min_run + 1) : p.workers;
   if (p.maxc > p.workers) p.maxc = p.workers;
+  if (p.m_tiles <= 4096) {  // the exact count: the most workers any range is split over
+    int mx = 1;
+    for (int64_t q = 0; q < p.m_tiles; ++q) {
+      const int lo = worker_of(q * p.upr, p.units, p.workers);
+      const int hi = worker_of(q * p.upr + p.upr - 1, p.units, p.workers);
+      mx = hi - lo + 1 > mx ? hi - lo + 1 : mx;
+    }
+    p.maxc = mx;
+  }
   // T slices: at most kGemvTSlices, a whole number of k blocks each
   p.bps = (p.kbt + kGemvTSlices - 1) / kGemvTSlices;
   p.t_slices = (p.kbt + p.bps - 1) / p.bps;
@@ -620,7 +632,7 @@ cudaError_t launch_gemv_mb(const GemvArgs& a, const GemvPlan& p, const uint16_t*
   if (a.M <= 8) err = launch_pdl(nf4_gemv_kernel<1>, dim3(p.grid), dim3(kGThreads), smem, st, args);
   else err = launch_pdl(nf4_gemv_kernel<2>, dim3(p.grid), dim3(kGThreads), smem, st, args);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(gemv_finish_kernel<MB>, dim3((unsigned)((a.N + 31) / 32)), dim3(128), 0, st, a.part, a.sTw, L2,
+  err = launch_pdl(gemv_finish_kernel<MB>, dim3((unsigned)((a.N + 31) / 32)), dim3(32 * kFinWarps), 0, st, a.part, a.sTw, L2,
                    a.M, a.N, a.r, p.upr, p.units, p.workers, p.maxc, Y);
   count_launches(3);
   return err != cudaSuccess ? err : cudaGetLastError();

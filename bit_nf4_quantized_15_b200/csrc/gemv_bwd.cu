@@ -546,13 +546,22 @@ GemvTPlan plan_gemv_t(int64_t M, int64_t N, int64_t K, int num_sms) {
   p.kbt = (int)(K / 64);
   p.k_ranges = (int)((K + 255) / 256);
   p.units = (int64_t)p.n_tiles * p.k_ranges;
-  // at least 4 units per worker (fewer partial tiles), at most one CTA per SM
-  const int64_t want = (p.units + kTG * 4 - 1) / (kTG * 4);
+  // at least 2 units per worker (fewer partial tiles to sum), at most one CTA per SM
+  const int64_t want = (p.units + kTG * 2 - 1) / (kTG * 2);
   p.grid = (int)(want < num_sms ? (want > 0 ? want : 1) : num_sms);
   p.workers = p.grid * kTG;
   const int64_t min_run = p.units / p.workers;
   p.maxc = min_run > 0 ? (int)((p.n_tiles + min_run - 1) / min_run + 1) : p.workers;
   if (p.maxc > p.workers) p.maxc = p.workers;
+  if (p.k_ranges <= 4096) {  // the exact count: the most workers any range is split over
+    int mx = 1;
+    for (int64_t q = 0; q < p.k_ranges; ++q) {
+      const int lo = t_worker_of(q * p.n_tiles, p.units, p.workers);
+      const int hi = t_worker_of(q * p.n_tiles + p.n_tiles - 1, p.units, p.workers);
+      mx = hi - lo + 1 > mx ? hi - lo + 1 : mx;
+    }
+    p.maxc = mx;
+  }
   // dT slices over N: at most 32, whole multiples of 8 columns
   int P = (int)((N + 255) / 256);
   if (P > 32) P = 32;
