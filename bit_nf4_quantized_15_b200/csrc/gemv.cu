@@ -251,8 +251,8 @@ __global__ void __launch_bounds__(kGThreads, 1) nf4_gemv_kernel(const __grid_con
 
   if (warp == 0) {
     // ------------------------------------ producers: one lane per ring stage
-    // (lane 2g + j fills stage j of worker g; a thread keeps about one
-    // large TMA box in flight at a time)
+    // (lane 2g + j fills stage j of worker g; they poll with a short sleep,
+    // so their turns in the warp cost nothing measurable here)
     if (lane < kWG * kWS) {
       const int g = lane / kWS, wk = c * kWG + g;
       const int64_t u0 = (int64_t)wk * U / W, u1 = (int64_t)(wk + 1) * U / W;
