@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
   constexpr int kStages = R::S;
   constexpr int kA = R::KA;
   constexpr int kCS = R::CS;
+  constexpr int kCSd = kCS ? kCS : 1;  // divisor for the code-ring index (dX only)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -261,8 +262,8 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
     // ----------------------------------------------- dX code-ring producer
     if (lane == 0 && !args.stall) {
       for (int it = 0; it < my_kb; ++it) {
-        const int c = it % kCS;
-        if (!mbar_wait(cempty + c, ((uint32_t)(it / kCS) & 1u) ^ 1u, abort_flag, args.status, lim)) break;
+        const int c = it % kCSd;
+        if (!mbar_wait(cempty + c, ((uint32_t)(it / kCSd) & 1u) ^ 1u, abort_flag, args.status, lim)) break;
         mbar_arrive_expect_tx(cfull + c, 4096u);
         tma_load_2d(smem + L::CODE + c * 4096, &args.tmA, cfull + c, row0 / 2, (kb_lo + it) * 64);
       }
@@ -365,8 +366,8 @@ __global__ void __launch_bounds__(Ring<AMODE>::THREADS, 1) umma_engine_kernel(co
         }
         const Nf4BlockTable tab = nf4_block_table(q, chat);
         // the codes first (their ring stage is freed once read), then the A buffer
-        const int c = it % kCS;
-        if (!warp_wait(cfull + c, (uint32_t)(it / kCS) & 1u, abort_flag, args.status, lane, lim)) break;
+        const int c = it % kCSd;
+        if (!warp_wait(cfull + c, (uint32_t)(it / kCSd) & 1u, abort_flag, args.status, lane, lim)) break;
         const uint8_t* ctile = smem + L::CODE + c * 4096 + nl * 64;
         uint4 cws[2];
 #pragma unroll
