@@ -53,7 +53,7 @@ WORKLOAD = "llama65b_block"
 # step: the mean over its 14 fused launches (Y and dX of the 7 linears) of
 # dram__bytes_read.sum + dram__bytes_write.sum, one single-pass ncu capture
 # of `bench.py --no-extras --no-cpu-baseline --steps 1 --warmup 1`.
-FUSED_TRAFFIC_BYTES = 913.4e6
+FUSED_TRAFFIC_BYTES = 907.0e6
 RT_WORKLOAD = ("bulk NF4 round trip of 2^31 bf16 weights (4 GiB): half N(0, 0.02), half Student-t(3) x 0.02 "
                "with 0.1% outliers x50; one launch per direction")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}

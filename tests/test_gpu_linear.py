@@ -208,6 +208,18 @@ def test_repeatable(lib):
         assert np.array_equal(a[k], b[k]), k
 
 
+def test_engine_repeatable_long_reduction(lib):
+    """The large-M engine, run three times on a long reduction (dX: 172
+    64-wide stages per tile through the four A buffers and the eight-stage
+    code ring), gives the same bits every time: a stage reused before its
+    readers are done would show up as a difference."""
+    case = make_case(1024, 11008, 2048, 64, seed=21)
+    runs = [run_gpu(lib, *case, 0.25) for _ in range(3)]
+    for k in runs[0]:
+        for other in runs[1:]:
+            assert np.array_equal(runs[0][k], other[k]), k
+
+
 # ------------------------------------------------------------- full sizes
 def _full_linear(q, wl, lin, M=None, sample_rows=64, seed=0):
     t = WL.make_linear(wl, lin, seed=seed, device="cpu", M=M)
