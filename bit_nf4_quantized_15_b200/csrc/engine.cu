@@ -3,15 +3,18 @@
 //   D[rows x cols] (fp32, in TMEM) = sum_k A[row, k] * B[col, k]
 //
 // One CTA computes a 128 x BN output tile with cta_group::1 UMMA (M = 128).
-// The reduction runs in 64-wide blocks through a 4-stage shared-memory ring:
+// The reduction runs in 64-wide blocks through a shared-memory ring (see
+// Ring for its depth per mode):
 //   * warp 0, one lane: TMA producer (B tiles, A tiles or NF4 code tiles),
-//     stages in order;
+//     stages in order; for dX a second producer warp fills a separate ring
+//     of code tiles;
 //   * warp 1, one lane: UMMA issuer, 4 x (128 x BN x 16) MMAs per stage,
 //     tcgen05.commit frees the stage;
-//   * warps 2..5 (128 threads): when A is the NF4 weight, they turn the code
-//     tile into a bf16 tile in the 128-byte-swizzled canonical layout UMMA
-//     reads (K-major for X.W^T, MN-major for dY.W), then run the epilogue
-//     (TMEM -> registers -> global, one accumulator row per thread).
+//   * dequant groups of 4 warps (128 threads): when A is the NF4 weight,
+//     they turn the code tile into a bf16 tile, in tensor memory for X.W^T
+//     or in the 128-byte-swizzled MN-major shared-memory layout for dY.W,
+//     then all groups run the epilogue (TMEM -> registers -> global, one
+//     accumulator row per thread).
 // An optional extension segment appends more reduction blocks from other
 // operands into the same accumulator: this is how the LoRA term s.T.L2
 // (forward) and s.dT.L1^T (backward) is added to the dequantised product.
@@ -32,8 +35,8 @@ constexpr int kRasterGroup = 4;  // column tiles per raster group (see the kerne
 // TMEM, so its stages hold only B and the codes (36 KB) and six of them fit:
 // deep enough to cover the TMA latency plus the dequant of a stage at the
 // tensor-bound pace.  Three dequant groups (stage s always served by group
-// s % 3).  dX and the plain GEMMs keep A in shared memory: four 52 KB stages,
-// four groups.
+// s % 3).  dX and the plain GEMMs keep A in shared memory: four stages of
+// A + B (48 KB at BN = 256), four groups (dX: group g owns stage g).
 //
 // dX keeps its code tiles in a ring of their own (CS stages of 4 KB, filled by
 // a second producer warp): a dequant group frees a code stage as soon as it
