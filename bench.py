@@ -17,7 +17,8 @@ Prints one JSON line (rank 0): whole-job algorithmic TFLOP/s of the step
 (4 M K N + 6 M r (K + N) per linear; no dequantisation work counted), plus
   e2e        the same metric through the C ABI with the step's activations
              copied host->device and the adapter gradients device->host
-             inside the timed region;
+             inside the timed region (the copies of later linears overlap
+             the computation of earlier ones, on a copy stream);
   roofline   the fused dequant-GEMM launches (Y of the forward, dX of the
              backward), timed live by events the library records around
              them on the launching stream, against the measured dense-bf16
@@ -315,9 +316,14 @@ class BlockStep:
         self.fused_bytes = sum(2 * nf4_bytes(l.N, l.K) + 2 * 2 * M * (l.K + l.N) + 2 * 2 * r * (l.K + l.N)
                                + 2 * 2 * M * r for l in wl.linears)
 
-    def step(self, events=None, exchange=False):
+    def step(self, events=None, exchange=False, before=None, after=None):
+        """One forward + backward of every linear; `before(i)` / `after(i)`
+        run around linear i (stream waits and event records of a caller that
+        feeds the inputs from the host)."""
         q, s = self.q, self.wl.s
         for i, L in enumerate(self.layers):
+            if before is not None:
+                before(i)
             if events is not None:
                 q.set_gemm_events(events[i][0], events[i][1])
             q.linear_fwd(L["X"], L["w"], L["L1"], L["L2"], s, ws=self.ws, Y=L["Y"], T=L["T"])
@@ -325,6 +331,8 @@ class BlockStep:
                 q.set_gemm_events(events[i][2], events[i][3])
             q.linear_bwd(L["dY"], L["X"], L["T"], L["w"], L["L1"], L["L2"], s, ws=self.ws,
                          dX=L["dX"], dL1=L["dL1"], dL2=L["dL2"])
+            if after is not None:
+                after(i)
         if exchange:
             self.grads.all_reduce()
 
@@ -665,11 +673,26 @@ def run_ours(args):
     h2d = sum(x.numel() * 2 + y.numel() * 2 for x, y in zip(hX, hdY))
     d2h = blk.grads.nbytes
 
+    # The step's inputs go up on a copy stream, linear by linear, while the
+    # earlier linears compute: linear i waits for its own inputs only, and its
+    # buffers are refilled for the next step once this step's linear i is done.
+    copy_stream = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in blk.layers]
+    done = [torch.cuda.Event() for _ in blk.layers]
+    begin = torch.cuda.Event()
+
     def e2e_step():
+        cur = torch.cuda.current_stream(dev)
+        begin.record(cur)                 # every copy of the step starts after the step does
+        copy_stream.wait_event(begin)
         for i, L in enumerate(blk.layers):
-            L["X"].copy_(hX[i], non_blocking=True)
-            L["dY"].copy_(hdY[i], non_blocking=True)
-        blk.step(exchange=world > 1)
+            copy_stream.wait_event(done[i])
+            with torch.cuda.stream(copy_stream):
+                L["X"].copy_(hX[i], non_blocking=True)
+                L["dY"].copy_(hdY[i], non_blocking=True)
+            ready[i].record(copy_stream)
+        blk.step(exchange=world > 1, before=lambda i: cur.wait_event(ready[i]),
+                 after=lambda i: done[i].record(cur))
         hG.copy_(blk.grads.flat, non_blocking=True)
 
     for _ in range(max(args.warmup, 1)):
